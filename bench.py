@@ -1,0 +1,350 @@
+#!/usr/bin/env python
+"""Throughput of the dynamic byte-chunking hot path on B200.
+
+One step = one pass of the whole path over one synthetic ByteFlow-shaped batch
+(8 rows x 8192 bytes x d = 256, bf16 AR(1) features, eps^2 = 0.5, K = 2048,
+16 upsampling bins): chunk_coding_rate -> chunk_topk_select -> chunk_gather ->
+chunk_upsample, all through the C ABI (libdbc.so) on one stream.
+
+Metric: sequence bytes per second (byte positions of the batch / step time).
+Timing: W untimed warm-up steps, then exactly K steps, each preceded (outside
+its timed interval) by a 256 MB write that flushes the 126 MB L2; CUDA events
+on the launching stream; barrier + synchronize around the timed loop; max over
+ranks.  Under torchrun each rank runs its own batch (weak scaling, no
+collective on the data path).
+
+``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "coding-rate chunker bytes/sec at B=8,T=8192,d=256,K=2048; % of roofline"
+UNIT = "bytes/s"
+WORKLOAD = ("byteflow-shaped: rows=8, T=8192, d=256, bf16 AR(1) rho=0.9 features, eps^2=0.5, "
+            "K=2048 (BOS + 2047 Top-K), gather, 16-bin upsample d_g=d_l=256, W_bin ~ N(0,1/d)")
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dbc", choices=["dbc", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_pipeline(w, rows):
+    """The float64 oracle over the given rows: dR (C, all host threads), Top-K, gather, upsample."""
+    from oracle.chunking import BIN_OFFSET, gather, topk_select_rows, upsample
+    from oracle.rank1 import dR_rank1
+    sub = np.asarray(rows)
+    offs = np.concatenate([[0], np.cumsum(w.lengths[sub])]).astype(np.int64)
+    H = np.concatenate([w.row(r) for r in sub])
+    dR = dR_rank1(H, offs, w.eps2)
+    idx, io = topk_select_rows(dR, offs, w.K[sub])
+    Z = gather(H, offs, idx, io)
+    W = w.f32("W_bin")
+    upsample(Z, H, offs, idx, io, W, BIN_OFFSET)
+    return int(offs[-1])
+
+
+def cpu_baseline(w):
+    t0 = time.perf_counter()
+    n = oracle_pipeline(w, range(w.rows))
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"whole batch ({w.rows} x {w.T} positions) through the float64 oracle: "
+                      f"rank-1 C recursion for dR on all host threads, Top-K, gather, upsample; {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import workloads
+    w = workloads.make("byteflow")
+    for i in range(args.warmup):
+        oracle_pipeline(w, [i % w.rows])
+    t0 = time.perf_counter()
+    n = 0
+    for i in range(args.steps):
+        n += oracle_pipeline(w, [i % w.rows])
+    dt = time.perf_counter() - t0
+    v = n / dt
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample_per_step": "one row (8192 positions)"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": "one 8192-position row per step through the float64 oracle"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- device arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import workloads
+    import dynamic_byte_chunking_b200 as dbc
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    stream = torch.cuda.current_stream()
+
+    w = workloads.make("byteflow", seed=1 + rank)
+    rows, T, d, K = w.rows, w.T, w.d, int(w.K[0])
+    N = w.N
+    H_host = torch.from_numpy(w.H_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    H = H_host.to(dev).view(rows, T, d)
+    Wb = torch.from_numpy(w.W_bin.view(np.int16)).view(torch.bfloat16).to(dev)
+    nb = Wb.shape[0]
+    dR = torch.empty(N, dtype=torch.float32, device=dev)
+    idx = torch.empty(rows * K, dtype=torch.int64, device=dev)
+    io = torch.empty(rows + 1, dtype=torch.int64, device=dev)
+    Z = torch.empty(rows * K, d, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(N, d, dtype=torch.float32, device=dev)
+    ws_cr = torch.empty(dbc.chunk_coding_rate_workspace(rows, T, N, d), dtype=torch.uint8, device=dev)
+    ws_up = torch.empty(dbc.chunk_upsample_workspace(rows, N, nb), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    stages = ["chunk_coding_rate", "chunk_topk_select", "chunk_gather", "chunk_upsample"]
+
+    def step(Hx, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dbc.chunk_coding_rate(Hx, w.eps2, dR=dR, workspace=ws_cr, dev_status=st)
+        if ev is not None:
+            ev[1].record(stream)
+        dbc.chunk_topk_select(dR, K, rows=rows, T=T, idx=idx, idx_offsets=io, dev_status=st)
+        if ev is not None:
+            ev[2].record(stream)
+        dbc.chunk_gather(Hx, idx, io, rows=rows, T=T, total=rows * K, Z=Z, dev_status=st)
+        if ev is not None:
+            ev[3].record(stream)
+        dbc.chunk_upsample(Z, Hx, idx, io, Wb, rows=rows, T=T, S=S, workspace=ws_up, dev_status=st)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(H)
+    torch.cuda.synchronize()
+    if st.item() != 0:
+        raise RuntimeError(f"device status flags {st.item():#x} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    gpu_id = str(local)
+    try:
+        props = torch.cuda.get_device_properties(dev)
+        if getattr(props, "uuid", None) is not None:
+            gpu_id = "GPU-" + str(props.uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = dbc.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        step(H, evs[k])
+    torch.cuda.synchronize()
+    launches = dbc.launch_count() - launches0
+    if pg:
+        pg.barrier()
+    time.sleep(0.2)
+    clocks = sampler.stop()
+
+    per_stage = np.zeros(4)
+    total = 0.0
+    for e in evs:
+        for s in range(4):
+            per_stage[s] += e[s].elapsed_time(e[s + 1])
+        total += e[0].elapsed_time(e[4])
+    t_ms = torch.tensor([total], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t_ms, op=pg.ReduceOp.MAX)
+    total_max = float(t_ms.item())
+    ms_per_step = total_max / args.steps
+    value = N * world / (ms_per_step * 1e-3)
+
+    # ---- roofline of the dominant stage (the coding-rate call)
+    pk, src = peaks()
+    avg = per_stage / args.steps          # ms per call
+    dom = int(np.argmax(avg))
+    flops_cr = 4.0 * d * d * N            # rank-1 recursion: 2d^2 (solve) + 2d^2 (update) per position
+    bytes_stage = [N * d * 2 + N * 4,                       # dR: read H, write dR
+                   N * 4 + rows * K * 8 + (rows + 1) * 8,   # Top-K: read dR, write idx
+                   2 * rows * K * d * 2,                    # gather: read + write chunk rows
+                   N * d * 2 + rows * K * d * 2 + nb * d * d * 2 + N * d * 4]  # upsample
+    if dom == 0:
+        achieved = flops_cr / (avg[0] * 1e-3) / 1e12
+        peak = pk.get("bf16_tflops_sustained", 1400.0)
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": stages[0],
+                "algorithmic": f"4*d^2*N = {flops_cr:.3e} flop per call", "peak_source": src + " sustained bf16"}
+    else:
+        achieved = bytes_stage[dom] / (avg[dom] * 1e-3) / 1e9
+        peak = pk.get("hbm_gbs", 6650.0)
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None, "kernel": stages[dom], "algorithmic": f"{bytes_stage[dom]} bytes per call",
+                "peak_source": src}
+
+    # ---- end to end through host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        out_idx = torch.empty(rows * K, dtype=torch.int64).pin_memory()
+        out_Z = torch.empty(rows * K, d, dtype=torch.bfloat16).pin_memory()
+        out_S = torch.empty(N, d, dtype=torch.float32).pin_memory()
+        Hdev = torch.empty(rows, T, d, dtype=torch.bfloat16, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            Hdev.copy_(H_host.view(rows, T, d), non_blocking=True)
+            step(Hdev)
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(args.e2e_steps):
+            flush.zero_()
+            e0.record(stream)
+            Hdev.copy_(H_host.view(rows, T, d), non_blocking=True)
+            step(Hdev)
+            out_idx.copy_(idx, non_blocking=True)
+            out_Z.copy_(Z, non_blocking=True)
+            out_S.copy_(S, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        te = torch.tensor([tot], dtype=torch.float64, device=dev)
+        if pg:
+            pg.all_reduce(te, op=pg.ReduceOp.MAX)
+        ms_e2e = float(te.item()) / args.e2e_steps
+        e2e = {"value": N * world / (ms_e2e * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(H_host.numel() * 2),
+               "d2h_bytes_per_step": int(out_idx.numel() * 8 + out_Z.numel() * 2 + out_S.numel() * 4),
+               "ms_per_step": ms_e2e}
+
+    torch.cuda.synchronize()
+    if st.item() != 0:
+        raise RuntimeError(f"device status flags {st.item():#x}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "rows_per_gpu": rows, "T": T, "d": d, "K": K, "nbins": nb,
+                           "global_batch": rows * world, "parallelism": f"dp{world} (independent rows)",
+                           "l2": "flushed by a 256 MB write before every timed step",
+                           "step": " -> ".join(stages)},
+                "stage_ms": {s: float(a) for s, a in zip(stages, avg)},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

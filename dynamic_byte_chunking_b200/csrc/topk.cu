@@ -1,0 +1,243 @@
+// chunk_topk_select: boundary positions per row.
+//
+// ByteFlow (papernotes.org notes, "Key design 2"; paper.rainbus.top summary,
+// "Method steps", stage 2): the first position is always a boundary, the K-1
+// positions with the largest dR among t >= 1 join it, and the K boundaries are
+// listed in time order.  Ties are broken towards the earlier position.
+//
+// One CTA per row: the row's dR values become order-preserving 32-bit keys
+// (in shared memory when they fit), a 4-pass 8-bit radix select finds the
+// (K-1)-th largest key v and how many keys equal to v are still needed, and
+// one ordered pass writes the selected positions, which are then already in
+// increasing order (no sort).
+#include "common.cuh"
+
+namespace dbc {
+namespace tk {
+
+constexpr int kThreads = 1024;
+constexpr int kSmemKeys = 48 * 1024;   // keys held in shared memory (192 KB)
+
+__device__ __forceinline__ uint32_t key_of(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u << 1) == 0u) u = 0u;                      // -0 and +0 are equal
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive block-wide scan of v over kThreads threads; *total gets the sum.
+__device__ __forceinline__ int block_excl_scan(int v, int *wsum, int *total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        int w = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        wsum[lane] = w;
+    }
+    __syncthreads();
+    const int r = (wid ? wsum[wid - 1] : 0) + x - v;
+    *total = wsum[31];
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ int64_t row_K(const int64_t *Kp, int64_t Ks, int64_t r, int32_t *st) {
+    int64_t K = Kp ? Kp[r] : Ks;
+    if (K < 1) {
+        flag(st, DBC_ERR_BOUNDS);
+        K = 1;
+    }
+    return K;
+}
+
+__global__ void __launch_bounds__(1024) offsets_kernel(const int64_t *offsets, int64_t rows, int64_t T,
+                                                       const int64_t *Kp, int64_t Ks,
+                                                       int64_t *idx_offsets, int32_t *st) {
+    __shared__ int64_t wsum[32];
+    __shared__ int64_t carry;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int64_t base = 0; base < rows; base += blockDim.x) {
+        const int64_t r = base + tid;
+        int64_t cnt = 0;
+        if (r < rows) {
+            int64_t a, n;
+            row_bounds(offsets, r, T, a, n);
+            const int64_t K = row_K(Kp, Ks, r, st);
+            cnt = n < K ? n : K;
+        }
+        int64_t x = cnt;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int64_t w = wsum[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            wsum[lane] = w;
+        }
+        __syncthreads();
+        const int64_t excl = carry + (wid ? wsum[wid - 1] : 0) + x - cnt;
+        if (r < rows) idx_offsets[r] = excl;
+        __syncthreads();
+        if (tid == (int)blockDim.x - 1) carry = excl + cnt;
+        __syncthreads();
+    }
+    if (tid == 0) idx_offsets[rows] = carry;
+}
+
+__global__ void __launch_bounds__(kThreads) select_kernel(const float *__restrict__ dR,
+                                                          const int64_t *offsets, int64_t rows, int64_t T,
+                                                          const int64_t *Kp, int64_t Ks,
+                                                          const int64_t *idx_offsets, int64_t *idx,
+                                                          int keys_in_smem, int32_t *st) {
+    extern __shared__ uint32_t keys[];
+    __shared__ uint32_t hist[256];
+    __shared__ int wsum[32];
+    __shared__ uint32_t s_bin;
+    __shared__ int64_t s_rem;
+    const int tid = threadIdx.x;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        int64_t a, n;
+        row_bounds(offsets, r, T, a, n);
+        const int64_t K = row_K(Kp, Ks, r, nullptr);
+        int64_t *out = idx + idx_offsets[r];
+        if (n <= 0) continue;
+        if (K >= n) {
+            for (int64_t t = tid; t < n; t += kThreads) out[t] = t;
+            continue;
+        }
+        if (tid == 0) out[0] = 0;
+        const int64_t need = K - 1;
+        if (need == 0) continue;
+        const int64_t m = n - 1;                 // candidates are t = 1 .. n-1
+        const float *row = dR + a + 1;
+        const bool in_smem = m <= keys_in_smem;
+        bool bad = false;
+        if (in_smem) {
+            for (int64_t j = tid; j < m; j += kThreads) {
+                const float f = row[j];
+                bad |= !isfinite(f);
+                keys[j] = key_of(f);
+            }
+        } else {
+            for (int64_t j = tid; j < m; j += kThreads) bad |= !isfinite(row[j]);
+        }
+        if (bad) flag(st, DBC_ERR_NONFINITE);
+        __syncthreads();
+        uint32_t prefix = 0, mask = 0;
+        int64_t rem = need;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int b = tid; b < 256; b += kThreads) hist[b] = 0;
+            __syncthreads();
+            for (int64_t j = tid; j < m; j += kThreads) {
+                const uint32_t k = in_smem ? keys[j] : key_of(row[j]);
+                if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (tid < 32) {
+                // warp 0: suffix sums over 8 bins per lane, then pick the bin
+                uint32_t c8[8];
+                uint32_t loc = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) { c8[q] = hist[255 - (tid * 8 + q)]; loc += c8[q]; }
+                uint32_t inc = loc;   // inclusive prefix over lanes (from the top bin down)
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (tid >= o) inc += y;
+                }
+                const uint32_t before = inc - loc;
+                const bool mine = (int64_t)before < rem && (int64_t)inc >= rem;
+                if (mine) {
+                    uint32_t cum = before;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if ((int64_t)(cum + c8[q]) >= rem) {
+                            s_bin = 255u - (uint32_t)(tid * 8 + q);
+                            s_rem = rem - (int64_t)cum;
+                            break;
+                        }
+                        cum += c8[q];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix |= s_bin << shift;
+            mask |= 255u << shift;
+            rem = s_rem;
+            __syncthreads();
+        }
+        // ordered compaction: key > v, or key == v among the first `rem` equal keys
+        const uint32_t v = prefix;
+        int64_t carry_eq = 0, carry_sel = 0;
+        for (int64_t base = 0; base < m; base += kThreads) {
+            const int64_t j = base + tid;
+            uint32_t k = 0;
+            if (j < m) k = in_smem ? keys[j] : key_of(row[j]);
+            const int eq = (j < m && k == v) ? 1 : 0;
+            int tot_eq;
+            const int eq_rank = block_excl_scan(eq, wsum, &tot_eq);
+            const int sel = (j < m && (k > v || (eq && carry_eq + eq_rank < rem))) ? 1 : 0;
+            int tot_sel;
+            const int pos = block_excl_scan(sel, wsum, &tot_sel);
+            if (sel) out[1 + carry_sel + pos] = j + 1;
+            carry_eq += tot_eq;
+            carry_sel += tot_sel;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace tk
+}  // namespace dbc
+
+using namespace dbc;
+
+extern "C" size_t chunk_topk_select_workspace(int64_t rows) {
+    (void)rows;
+    return 0;
+}
+
+extern "C" dbc_status chunk_topk_select(const float *dR, const int64_t *offsets, int64_t rows,
+                                        int64_t T, int64_t N, const int64_t *K_per_row,
+                                        int64_t K_scalar, int64_t *idx, int64_t *idx_offsets,
+                                        void *ws, size_t ws_bytes, int32_t *dev_status,
+                                        dbc_stream_t stream) {
+    (void)ws; (void)ws_bytes;
+    if (rows < 0 || T < 0 || N < 0) return DBC_ERR_INVALID_ARG;
+    if (!K_per_row && K_scalar < 1) return DBC_ERR_INVALID_ARG;
+    if (!offsets && N != rows * T) return DBC_ERR_INVALID_ARG;
+    if (!idx_offsets) return DBC_ERR_INVALID_ARG;
+    if (rows > 0 && N > 0 && (!dR || !idx)) return DBC_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    tk::offsets_kernel<<<1, 1024, 0, s>>>(offsets, rows, T, K_per_row, K_scalar, idx_offsets,
+                                          dev_status);
+    count_launches(1);
+    if (rows == 0 || N == 0) return launch_status();
+    const int64_t m = T > 1 ? T - 1 : 1;
+    const int keys = (int)std::min<int64_t>(m, tk::kSmemKeys);
+    const size_t smem = (size_t)keys * sizeof(uint32_t);
+    cudaFuncSetAttribute(tk::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int grid = (int)std::min<int64_t>(rows, 65535);
+    tk::select_kernel<<<grid, tk::kThreads, smem, s>>>(dR, offsets, rows, T, K_per_row, K_scalar,
+                                                       idx_offsets, idx, keys, dev_status);
+    count_launches(1);
+    return launch_status();
+}

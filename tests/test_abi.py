@@ -1,0 +1,72 @@
+"""The C-ABI library loads on a CPU-only host and exports every declared entry point.
+
+No kernel is launched here: only symbol lookup, status names, the version and
+the host-side workspace queries, which need no device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dbc.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"DBC_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import dynamic_byte_chunking_b200 as dbc
+    from dynamic_byte_chunking_b200 import build
+    build.build()
+    return dbc.lib()
+
+
+def test_header_declares_the_five_entry_points():
+    names = _declared()
+    for n in ("chunk_coding_rate", "chunk_topk_select", "chunk_gather", "chunk_upsample", "hnet_route"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in _declared():
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    import dynamic_byte_chunking_b200 as dbc
+    assert dbc.status_string(0) == "DBC_OK"
+    assert dbc.status_string(7) == "DBC_ERR_WORKSPACE"
+    assert dbc.version() >= 100
+
+
+def test_workspace_queries_scale(L):
+    import dynamic_byte_chunking_b200 as dbc
+    a = dbc.chunk_coding_rate_workspace(8, 8192, 8 * 8192, 256)
+    b = dbc.chunk_coding_rate_workspace(16, 8192, 16 * 8192, 256)
+    assert 0 < a < b
+    assert dbc.chunk_upsample_workspace(8, 65536, 16) > 65536
+    assert dbc.hnet_route_workspace(64, 4096 * 64, 256) >= 4096 * 64 * 512 * 4
+
+
+def test_argument_errors_return_before_launch(L):
+    # Host-side validation runs before any CUDA call, so it works without a GPU.
+    f = L.chunk_coding_rate
+    # eps2 <= 0
+    assert f(None, 1, None, 1, 64, 64, 64, ctypes.c_float(0.0), None, None, 0, None, None) == 1
+    # unsupported width
+    assert f(None, 1, None, 1, 64, 64, 96, ctypes.c_float(0.5), None, None, 0, None, None) == 2
+    # dense N mismatch
+    assert f(None, 1, None, 2, 64, 64, 64, ctypes.c_float(0.5), None, None, 0, None, None) == 1
+    # empty batch is a no-op success
+    assert f(None, 1, None, 0, 64, 0, 64, ctypes.c_float(0.5), None, None, 0, None, None) == 0
+    # K < 1
+    assert L.chunk_topk_select(None, None, 1, 8, 8, None, 0, None, None, None, 0, None, None) == 1
+    # bad bin count / mode
+    u = L.chunk_upsample
+    assert u(None, 64, None, 1, None, 8, 8, 64, None, None, 1, None, 0, 0, None, None, 0, None, None) == 1
+    assert u(None, 64, None, 1, None, 8, 8, 64, None, None, 1, None, 16, 7, None, None, 0, None, None) == 1
