@@ -24,7 +24,7 @@ from typing import Optional
 __all__ = [
     "DbcError", "lib", "lib_path", "version", "status_string", "launch_count",
     "chunk_coding_rate", "chunk_coding_rate_workspace", "chunk_topk_select",
-    "chunk_gather", "chunk_upsample", "chunk_upsample_workspace",
+    "chunk_gather", "chunk_upsample", "chunk_upsample_workspace", "chunk_upsample_noalloc",
     "hnet_route", "hnet_route_workspace", "chunk",
     "DBC_F32", "DBC_BF16", "BIN_OFFSET", "BIN_FRACTION", "BIN_ABSOLUTE",
     "ERR_NONFINITE", "ERR_TIMEOUT", "ERR_BOUNDS",
@@ -53,6 +53,8 @@ _SIGS = {
     "chunk_upsample_workspace": (_sz, [_i64, _i64, _int]),
     "chunk_upsample": (_int, [_vp, _i64, _vp, _int, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _int,
                               _int, _vp, _vp, _sz, _vp, _vp]),
+    "chunk_upsample_noalloc": (_int, [_vp, _i64, _vp, _int, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp,
+                                      _int, _int, _vp, _vp, _vp]),
     "hnet_route_workspace": (_sz, [_i64, _i64, _i64]),
     "hnet_route": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _f32, _int, _vp, _vp, _vp, _vp,
                           _vp, _vp, _sz, _vp, _vp]),
@@ -251,6 +253,24 @@ def chunk_upsample(G, H, idx, idx_offsets, W_bin, *, rows: int, T: int, offsets=
                               _ptr(idx), _ptr(idx_offsets), rows, _ptr(W_bin.contiguous()), nbins, int(mode),
                               _ptr(S), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
     _check("chunk_upsample", rc)
+    return S
+
+
+def chunk_upsample_noalloc(G, H, idx, idx_offsets, W_bin, *, rows: int, T: int, offsets=None,
+                           mode: int = BIN_OFFSET, S=None, dev_status=None, stream=None):
+    """chunk_upsample without a workspace: scratch comes from the library's static
+    device array (N <= 1048576; calls that overlap on one device race on it)."""
+    torch = _torch()
+    _require_cuda(G, H, idx, idx_offsets, W_bin, offsets)
+    H2 = H.reshape(-1, H.shape[-1]).contiguous()
+    N, d_l = H2.shape
+    nbins, d_g, _ = W_bin.shape
+    if S is None:
+        S = torch.empty(N, d_l, dtype=torch.float32, device=H.device)
+    rc = lib().chunk_upsample_noalloc(_ptr(G.contiguous()), d_g, _ptr(H2), _dtype_code(H2), _ptr(offsets), T,
+                                      N, d_l, _ptr(idx), _ptr(idx_offsets), rows, _ptr(W_bin.contiguous()),
+                                      nbins, int(mode), _ptr(S), _ptr(dev_status), _stream(stream))
+    _check("chunk_upsample_noalloc", rc)
     return S
 
 

@@ -226,3 +226,86 @@ extern "C" dbc_status chunk_upsample(const void *G, int64_t d_g, const void *H, 
     count_launches(4);
     return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// chunk_upsample_noalloc: the same computation as chunk_upsample, for callers
+// that cannot hand the library a workspace.  Its scratch (per-position chunk
+// and bin, the bin permutation and the bin counters) lives in one file-scope
+// device array that every GPU loading this library holds until the process
+// exits.  Host code never passes that array's name to a kernel (in host code
+// it is only a stand-in for the device symbol); the device address is looked
+// up once per device with cudaGetSymbolAddress and cached.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace dbc {
+namespace up {
+
+constexpr int64_t kNoAllocMaxN = 1 << 20;                 // positions per call
+constexpr size_t kNoAllocScratchBytes = 10u << 20;        // 10 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_ptr[kNoAllocMaxDevices];
+
+// Device address of the static scratch on the current device (looked up on
+// the first call made with that device current, then cached).
+static dbc_status noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DBC_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return DBC_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DBC_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return DBC_OK;
+}
+
+}  // namespace up
+}  // namespace dbc
+
+extern "C" dbc_status chunk_upsample_noalloc(const void *G, int64_t d_g, const void *H, int dtype,
+                                             const int64_t *offsets, int64_t T, int64_t N, int64_t d_l,
+                                             const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
+                                             const void *W_bin, int nbins, int mode, float *S,
+                                             int32_t *dev_status, dbc_stream_t stream) {
+    if (rows < 0 || T < 0 || N < 0 || d_g <= 0 || d_l <= 0) return DBC_ERR_INVALID_ARG;
+    if (nbins < 1 || nbins > up::kMaxBins) return DBC_ERR_INVALID_ARG;
+    if (mode < DBC_BIN_IN_CHUNK_OFFSET || mode > DBC_BIN_ABSOLUTE) return DBC_ERR_INVALID_ARG;
+    if (dtype != DBC_F32 && dtype != DBC_BF16) return DBC_ERR_UNSUPPORTED;
+    if (d_g % 64 || d_l % 64 || d_g > 2048 || d_l > 2048) return DBC_ERR_UNSUPPORTED;
+    if (!offsets && N != rows * T) return DBC_ERR_INVALID_ARG;
+    if (N > up::kNoAllocMaxN) return DBC_ERR_WORKSPACE;   // larger than the built-in scratch
+    if (N == 0 || rows == 0) return DBC_OK;
+    if (!G || !H || !idx || !idx_offsets || !W_bin || !S) return DBC_ERR_INVALID_ARG;
+    if (up::carve(nullptr, N).bytes > up::kNoAllocScratchBytes) return DBC_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    const dbc_status ss = up::noalloc_scratch(&scratch);
+    if (ss != DBC_OK) return ss;
+    const up::Layout L = up::carve(scratch, N);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The bin counters must start at zero; everything else is written before it is read.
+    cudaMemsetAsync(L.hist, 0, sizeof(int32_t) * up::kMaxBins, s);
+    const int sms = num_sms();
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (int64_t)sms * 8));
+    up::classify_kernel<<<grid, 256, 0, s>>>(offsets, T, N, idx, idx_offsets, rows, nbins, mode, L,
+                                             dev_status);
+    up::scan_bins_kernel<<<1, 32, 0, s>>>(nbins, L);
+    up::scatter_kernel<<<grid, 256, 0, s>>>(N, L);
+    dim3 g((unsigned)((N + 63) / 64 + nbins), (unsigned)(d_l / 64));
+    if (dtype == DBC_BF16)
+        up::bin_gemm_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
+            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S);
+    else
+        up::bin_gemm_kernel<float><<<g, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
+            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S);
+    count_launches(4);
+    return launch_status();
+}

@@ -173,6 +173,37 @@ DBC_API dbc_status chunk_upsample(const void *G, int64_t d_g, const void *H, int
                           dbc_stream_t stream);
 
 /* -------------------------------------------------------------------------
+ * chunk_upsample_noalloc -- chunk_upsample for callers that cannot allocate.
+ *
+ * No passage of the pages corresponds to this entry point; it is a deployment
+ * convenience.  Some callers cannot provide device scratch: a host thread
+ * inside an inference server whose device memory is entirely owned by the
+ * server's own pool, or a plugin/extension point that receives only its input
+ * and output buffers and must not call cudaMalloc (which can synchronise the
+ * device and fails once the memory budget is taken).  This variant computes
+ * exactly what chunk_upsample computes, with the same arguments minus the
+ * workspace, and calls no allocating routine (no cudaMalloc/cudaFree, no
+ * allocating library call).
+ *
+ * Its scratch is a built-in static device array of 10 MiB that every GPU
+ * loading libdbc.so keeps until the process exits.  Limit: N <= 1048576
+ * positions per call; larger N returns DBC_ERR_WORKSPACE before any launch
+ * (use chunk_upsample with a caller workspace instead).
+ * The first call made with a given device current looks up the array's device
+ * address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture.  All calls share the one array, which keeps the last
+ * call's contents (the call clears what must start at zero): calls that can
+ * overlap on the GPU -- concurrent streams or host threads on one device --
+ * race on it and must be serialised by the caller.
+ * Errors: as chunk_upsample, with DBC_ERR_WORKSPACE for N above the limit.
+ * ------------------------------------------------------------------------- */
+DBC_API dbc_status chunk_upsample_noalloc(const void *G, int64_t d_g, const void *H, int dtype,
+                                          const int64_t *offsets, int64_t T, int64_t N, int64_t d_l,
+                                          const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
+                                          const void *W_bin, int nbins, int mode, float *S,
+                                          int32_t *dev_status, dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
  * hnet_route -- cosine-similarity boundary router with EMA smoothing.
  *
  * ByteGen report ("H-Net architecture", "Methodology"): boundary probability
