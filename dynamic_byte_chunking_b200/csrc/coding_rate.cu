@@ -28,6 +28,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace dbc {
 namespace cr {
@@ -194,6 +195,131 @@ __global__ void __launch_bounds__(256) gram_kernel(const IN *__restrict__ H, int
 #pragma unroll
         for (int r = 0; r < 4; ++r)
             G[(size_t)(I * 64 + ty * 4 + q) * d + J * 64 + tx * 4 + r] = acc[q][r];
+}
+
+// ---------------------------------------------------------------- gram (tensor cores)
+// G_s = X_s^T X_s on tcgen05 (bf16 x bf16 products are exact, fp32 accumulation
+// in TMEM).  A 64-position chunk of X_s is staged once in shared memory as an
+// MN-major 128-byte-swizzled tile and read as both operands (A = features of
+// this CTA's 128-row blocks, B = all d features).  Three stages keep the next
+// cp.async fills in flight while the tensor core works on the current chunk.
+// grid (segment, row-block group), 128 threads.
+template <int D>
+struct GramTC {
+    static constexpr int NMB = (D == 256) ? 2 : 1;       // 128-row blocks per CTA
+    static constexpr int GROUPS = (D / 128) / NMB;       // CTAs per segment
+    static constexpr int NCOLS = NMB * D;                // TMEM columns used
+    static constexpr int TMEM_COLS = NCOLS <= 128 ? 128 : (NCOLS <= 256 ? 256 : 512);
+    static constexpr int KC = 64;                        // positions per chunk
+    static constexpr uint32_t LBO = KC * 128;            // bytes of one 64-feature block
+    static constexpr uint32_t STAGE = (D / 64) * LBO;
+    static constexpr int NS = 3;
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1) gram_tc_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+                                                          float *aug, int32_t *st) {
+    using C = GramTC<D>;
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[C::NS];
+    __shared__ uint32_t tmem_base;
+    const int s = blockIdx.x;
+    if (s >= *S.nseg) return;
+    const int mb0 = blockIdx.y * C::NMB;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int len = S.len[s];
+    const int64_t start = S.start[s];
+    const uint32_t raw = tc::smem_u32(smraw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, C::TMEM_COLS);
+    if (tid == 0) {
+        for (int i = 0; i < C::NS; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    const int nchunks = (len + C::KC - 1) / C::KC;
+    constexpr int F8 = D / 8;                            // 16-byte groups per position
+
+    auto load = [&](int c) {
+        const uint32_t sb = base + (uint32_t)(c % C::NS) * C::STAGE;
+        const int t0 = c * C::KC;
+        for (int e = tid; e < C::KC * F8; e += 128) {
+            const int p = e / F8, f8 = e - (e / F8) * F8;
+            const int pos = t0 + p;
+            const __nv_bfloat16 *src = H + (start + (pos < len ? pos : 0)) * D + f8 * 8;
+            tc::cp_async16(sb + tc::mnmajor_off(f8 * 8, p, C::LBO), src, pos < len ? 16u : 0u);
+        }
+        tc::cp_async_commit();
+    };
+
+    bool ok = true;
+    for (int c = 0; c < C::NS - 1; ++c) {
+        if (c < nchunks) load(c); else tc::cp_async_commit();
+    }
+    constexpr uint32_t idesc = tc::idesc_bf16(128, D < 256 ? D : 256, true, true);
+    for (int c = 0; c < nchunks; ++c) {
+        const int cn = c + C::NS - 1;
+        if (cn < nchunks) {
+            if (cn >= C::NS) ok &= tc::mbar_wait(&mbar[cn % C::NS], (uint32_t)((cn / C::NS) - 1) & 1u, st);
+            load(cn);
+        } else {
+            tc::cp_async_commit();
+        }
+        tc::cp_async_wait<C::NS - 1>();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t sb = base + (uint32_t)(c % C::NS) * C::STAGE;
+#pragma unroll
+            for (int kk = 0; kk < C::KC / 16; ++kk) {
+#pragma unroll
+                for (int m = 0; m < C::NMB; ++m) {
+                    const uint64_t ad = tc::sdesc(sb + (uint32_t)(2 * (mb0 + m)) * C::LBO + kk * 2048, C::LBO, 1024);
+#pragma unroll
+                    for (int nb = 0; nb < (D + 255) / 256; ++nb) {
+                        const uint64_t bd = tc::sdesc(sb + (uint32_t)(4 * nb) * C::LBO + kk * 2048, C::LBO, 1024);
+                        tc::mma_bf16(tbase + (uint32_t)(m * D + nb * 256), ad, bd, idesc,
+                                     (c > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+            }
+            tc::mma_commit(&mbar[c % C::NS]);
+        }
+        __syncthreads();
+    }
+    if (nchunks > 0) ok &= tc::mbar_wait(&mbar[(nchunks - 1) % C::NS], (uint32_t)((nchunks - 1) / C::NS) & 1u, st);
+    ok = __syncthreads_and(ok) != 0;      // the warp-collective TMEM loads below need a uniform decision
+    tc::fence_after_sync();
+    float *G = aug + (size_t)s * (size_t)(D + kSegMax) * (size_t)D;
+    bool bad = false;
+    if (ok) {
+#pragma unroll 1
+        for (int m = 0; m < C::NMB; ++m) {
+            const int row = (mb0 + m) * 128 + warp * 32 + lane;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)(m * D + c0), v);
+                if (nchunks == 0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                }
+                if (row >= c0 && row < c0 + 16) bad |= !isfinite(v[row - c0]);
+                float4 *dst = reinterpret_cast<float4 *>(G + (size_t)row * D + c0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+    }
+    if (bad) flag(st, DBC_ERR_NONFINITE);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, C::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- prefix
@@ -418,6 +544,31 @@ __global__ void __launch_bounds__(256) first_seg_kernel(const IN *__restrict__ H
     }
 }
 
+template <int D>
+void launch_gram_tc(const __nv_bfloat16 *H, int64_t ns, const Layout &L, int32_t *st, cudaStream_t stream) {
+    using C = GramTC<D>;
+    cudaFuncSetAttribute(gram_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    gram_tc_kernel<D><<<dim3((unsigned)ns, (unsigned)C::GROUPS), 128, C::SMEM, stream>>>(H, L.segs, L.aug, st);
+}
+
+inline void launch_gram(const float *H, int64_t d, int64_t ns, const Layout &L, int32_t *st,
+                        cudaStream_t stream) {
+    gram_kernel<float><<<dim3((unsigned)ns, (unsigned)((d / 64) * (d / 64))), 256, 0, stream>>>(
+        H, d, L.segs, L.aug, st);
+}
+
+inline void launch_gram(const __nv_bfloat16 *H, int64_t d, int64_t ns, const Layout &L, int32_t *st,
+                        cudaStream_t stream) {
+    switch (d) {
+        case 128: launch_gram_tc<128>(H, ns, L, st, stream); return;
+        case 256: launch_gram_tc<256>(H, ns, L, st, stream); return;
+        case 512: launch_gram_tc<512>(H, ns, L, st, stream); return;
+        default:
+            gram_kernel<__nv_bfloat16><<<dim3((unsigned)ns, (unsigned)((d / 64) * (d / 64))), 256, 0, stream>>>(
+                H, d, L.segs, L.aug, st);
+    }
+}
+
 template <class IN>
 dbc_status run(const IN *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N, int64_t d,
                float eps2, float *dR, const Layout &L, int32_t *st, cudaStream_t stream) {
@@ -425,8 +576,7 @@ dbc_status run(const IN *H, const int64_t *offsets, int64_t rows, int64_t T, int
     const int64_t ns = nseg_upper(rows, N);
     const int sms = num_sms();
     seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, L.segs, st);
-    gram_kernel<IN><<<dim3((unsigned)ns, (unsigned)((d / 64) * (d / 64))), 256, 0, stream>>>(
-        H, d, L.segs, L.aug, st);
+    launch_gram(H, d, ns, L, st, stream);
     prefix_kernel<<<dim3((unsigned)rows, (unsigned)((d * d + 255) / 256)), 256, 0, stream>>>(
         L.segs, L.aug, d, c);
     fill_x_kernel<IN><<<dim3((unsigned)ns, 16), 256, 0, stream>>>(H, d, L.segs, L.aug);
