@@ -219,7 +219,7 @@ struct GramTC {
 
 template <int D>
 __global__ void __launch_bounds__(128, 1) gram_tc_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
-                                                          float *aug, int32_t *st) {
+                                                          float *aug, size_t mat_stride, int32_t *st) {
     using C = GramTC<D>;
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[C::NS];
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(128, 1) gram_tc_kernel(const __nv_bfloat16 *__
     if (nchunks > 0) ok &= tc::mbar_wait(&mbar[(nchunks - 1) % C::NS], (uint32_t)((nchunks - 1) / C::NS) & 1u, st);
     ok = __syncthreads_and(ok) != 0;      // the warp-collective TMEM loads below need a uniform decision
     tc::fence_after_sync();
-    float *G = aug + (size_t)s * (size_t)(D + kSegMax) * (size_t)D;
+    float *G = aug + (size_t)s * mat_stride;
     bool bad = false;
     if (ok) {
 #pragma unroll 1
@@ -509,20 +509,21 @@ __global__ void __launch_bounds__(256) first_seg_kernel(const IN *__restrict__ H
                                                         double c, float *dR) {
     extern __shared__ double sm1[];
     double *G = sm1;                                   // 64 x 65
-    float *X = reinterpret_cast<float *>(sm1 + 64 * 65);  // len x d
+    float *X = reinterpret_cast<float *>(sm1 + 64 * 65);  // len x (d + 1), padded rows
+    const int64_t ldx = d + 1;
     const int tid = threadIdx.x;
     const int nseg = *S.nseg;
     for (int s = blockIdx.x; s < nseg; s += gridDim.x) {
         if (S.k[s] != 0) continue;
         const int len = S.len[s];
         const int64_t start = S.start[s];
-        for (int64_t e = tid; e < (int64_t)len * d; e += 256) X[e] = ld_f(H + start * d + e);
+        for (int64_t e = tid; e < (int64_t)len * d; e += 256) X[(e / d) * ldx + (e % d)] = ld_f(H + start * d + e);
         __syncthreads();
         for (int e = tid; e < len * len; e += 256) {
             const int i = e / len, j = e - (e / len) * len;
             if (j <= i) {
                 double acc = 0.0;
-                for (int k = 0; k < d; ++k) acc += (double)X[i * d + k] * (double)X[j * d + k];
+                for (int k = 0; k < d; ++k) acc += (double)X[i * ldx + k] * (double)X[j * ldx + k];
                 G[i * 65 + j] = c * acc;
             }
         }
@@ -545,10 +546,12 @@ __global__ void __launch_bounds__(256) first_seg_kernel(const IN *__restrict__ H
 }
 
 template <int D>
-void launch_gram_tc(const __nv_bfloat16 *H, int64_t ns, const Layout &L, int32_t *st, cudaStream_t stream) {
+void launch_gram_tc(const __nv_bfloat16 *H, int64_t ns, const Segs &segs, float *mats, size_t mat_stride,
+                    int32_t *st, cudaStream_t stream) {
     using C = GramTC<D>;
     cudaFuncSetAttribute(gram_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    gram_tc_kernel<D><<<dim3((unsigned)ns, (unsigned)C::GROUPS), 128, C::SMEM, stream>>>(H, L.segs, L.aug, st);
+    gram_tc_kernel<D><<<dim3((unsigned)ns, (unsigned)C::GROUPS), 128, C::SMEM, stream>>>(H, segs, mats,
+                                                                                       mat_stride, st);
 }
 
 inline void launch_gram(const float *H, int64_t d, int64_t ns, const Layout &L, int32_t *st,
@@ -559,10 +562,11 @@ inline void launch_gram(const float *H, int64_t d, int64_t ns, const Layout &L, 
 
 inline void launch_gram(const __nv_bfloat16 *H, int64_t d, int64_t ns, const Layout &L, int32_t *st,
                         cudaStream_t stream) {
+    const size_t stride = (size_t)(d + kSegMax) * (size_t)d;
     switch (d) {
-        case 128: launch_gram_tc<128>(H, ns, L, st, stream); return;
-        case 256: launch_gram_tc<256>(H, ns, L, st, stream); return;
-        case 512: launch_gram_tc<512>(H, ns, L, st, stream); return;
+        case 128: launch_gram_tc<128>(H, ns, L.segs, L.aug, stride, st, stream); return;
+        case 256: launch_gram_tc<256>(H, ns, L.segs, L.aug, stride, st, stream); return;
+        case 512: launch_gram_tc<512>(H, ns, L.segs, L.aug, stride, st, stream); return;
         default:
             gram_kernel<__nv_bfloat16><<<dim3((unsigned)ns, (unsigned)((d / 64) * (d / 64))), 256, 0, stream>>>(
                 H, d, L.segs, L.aug, st);
@@ -588,7 +592,7 @@ dbc_status run(const IN *H, const int64_t *offsets, int64_t rows, int64_t T, int
     chol_kernel<false><<<chol_grid, 256, smem_f, stream>>>(L.segs, L.aug, L.gp, d, dR);
     ygram_kernel<<<dim3((unsigned)ns, 36), 256, 0, stream>>>(L.segs, L.aug, d, (float)c, L.gp);
     chol_kernel<true><<<chol_grid, 256, smem_i, stream>>>(L.segs, L.aug, L.gp, d, dR);
-    const size_t smem1 = 64 * 65 * sizeof(double) + (size_t)64 * d * sizeof(float);
+    const size_t smem1 = 64 * 65 * sizeof(double) + (size_t)64 * (d + 1) * sizeof(float);
     cudaFuncSetAttribute(first_seg_kernel<IN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
     first_seg_kernel<IN><<<(unsigned)std::min<int64_t>(ns, (int64_t)sms * 2), 256, smem1, stream>>>(
         H, d, L.segs, c, dR);
@@ -599,12 +603,19 @@ dbc_status run(const IN *H, const int64_t *offsets, int64_t rows, int64_t T, int
 }  // namespace cr
 }  // namespace dbc
 
+#include "segment_tc.cuh"
+
 using namespace dbc;
+
+static bool use_tensor_path(int dtype, int64_t d) {
+    return dtype == DBC_BF16 && (d == 128 || d == 256 || d == 512);
+}
 
 extern "C" size_t chunk_coding_rate_workspace(int64_t rows, int64_t T, int64_t N, int64_t d) {
     (void)T;
     if (rows < 0 || N < 0 || d <= 0) return 0;
-    return cr::carve(nullptr, rows, N, d).bytes;
+    // large enough for either path (the dtype is not an argument of the query)
+    return std::max(cr::carve(nullptr, rows, N, d).bytes, cr::carve2(nullptr, rows, N, d).bytes);
 }
 
 extern "C" dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t *offsets,
@@ -618,11 +629,23 @@ extern "C" dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t 
     if (N == 0 || rows == 0) return DBC_OK;
     if (!H || !dR || !aligned16(H)) return DBC_ERR_INVALID_ARG;
     if (cr::nseg_upper(rows, N) > INT32_MAX / 2) return DBC_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_tensor_path(dtype, d)) {
+        const cr::Layout2 need2 = cr::carve2(nullptr, rows, N, d);
+        if (!ws || ws_bytes < need2.bytes || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)))
+            return DBC_ERR_WORKSPACE;
+        const cr::Layout2 L2 = cr::carve2(ws, rows, N, d);
+        const __nv_bfloat16 *Hb = static_cast<const __nv_bfloat16 *>(H);
+        switch (d) {
+            case 128: return cr::run_tc<128>(Hb, offsets, rows, T, N, eps2, dR, L2, dev_status, s);
+            case 256: return cr::run_tc<256>(Hb, offsets, rows, T, N, eps2, dR, L2, dev_status, s);
+            default: return cr::run_tc<512>(Hb, offsets, rows, T, N, eps2, dR, L2, dev_status, s);
+        }
+    }
     const cr::Layout need = cr::carve(nullptr, rows, N, d);
     if (!ws || ws_bytes < need.bytes || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)))
         return DBC_ERR_WORKSPACE;
     const cr::Layout L = cr::carve(ws, rows, N, d);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == DBC_BF16)
         return cr::run(static_cast<const __nv_bfloat16 *>(H), offsets, rows, T, N, d, eps2, dR, L,
                        dev_status, s);

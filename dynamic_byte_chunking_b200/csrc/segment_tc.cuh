@@ -1,0 +1,416 @@
+// Coding-rate segments on tensor cores (bf16 features, d in {128, 256, 512}).
+// Included by coding_rate.cu, which holds the segment table, the tcgen05
+// Gram and the float64 first-segment kernel this path shares.
+//
+// Per segment s (rows X_s, start state M_s = I + P_s):
+//   factor: panel Cholesky of [P_s ; I] with the identity implicit; the
+//           appended block becomes B = L_s^{-T} (L_s L_s^T = M_s);
+//   ainv:   A_s = B B^T = M_s^{-1}, stored as three bf16 pieces (hi, mid, lo)
+//           whose sum carries the fp32 value;
+//   vgemm:  V = X_s A_s on tcgen05 (X exact in bf16, three passes over the
+//           pieces, fp32 accumulation in TMEM); V stored as three pieces;
+//   kgemm:  G'_s = c X_s V^T on tcgen05 (three passes), lower 128-blocks;
+//   inseg:  panel Cholesky of I + G'_s with the identity implicit; the
+//           excess e_t of each diagonal gives dR_t = log1p(e_t) / 2.
+// G'_s = c X_s M_s^{-1} X_s^T is the in-segment Gram in the frame whitened
+// by the segment's start state, so its Cholesky diagonal is the per-position
+// Schur complement 1 + c h_t^T M_{t-1}^{-1} h_t (matrix determinant lemma).
+#pragma once
+
+#include "panel_chol.cuh"
+#include "tc.cuh"
+
+namespace dbc {
+namespace cr {
+
+struct Layout2 {
+    Segs segs;
+    float *aug2;            // per segment: [2D][D] = [P_s ; I] -> [. ; L^{-T}]
+    __nv_bfloat16 *A3;      // per segment: [3][D][D]
+    __nv_bfloat16 *V3;      // [3][N][D]
+    float *gp;              // per segment at start*kSegMax: len x ldg(len)
+    size_t bytes;
+};
+
+__host__ __device__ inline int ldg_of(int len) { return (len + 3) & ~3; }
+
+inline Layout2 carve2(void *ws, int64_t rows, int64_t N, int64_t d) {
+    Carver c(ws);
+    const int64_t ns = nseg_upper(rows, N);
+    Layout2 L;
+    L.segs.start = c.take<int64_t>(ns);
+    L.segs.len = c.take<int32_t>(ns);
+    L.segs.row = c.take<int32_t>(ns);
+    L.segs.k = c.take<int32_t>(ns);
+    L.segs.row_seg0 = c.take<int32_t>(rows + 1);
+    L.segs.nseg = c.take<int32_t>(1);
+    L.aug2 = c.take<float>((size_t)ns * 2 * d * d);
+    L.A3 = c.take<__nv_bfloat16>((size_t)ns * 3 * d * d);
+    L.V3 = c.take<__nv_bfloat16>((size_t)3 * N * d + 8);
+    L.gp = c.take<float>((size_t)N * kSegMax + 4);
+    L.bytes = c.off;
+    return L;
+}
+
+// ---------------------------------------------------------------- prefix
+// In place over a row's segments: Gram -> P_s = c sum_{s'<s} G_s' (float64
+// running sum, fp32 store); the appended block of each matrix becomes I.
+__global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c) {
+    const int64_t r = blockIdx.x;
+    const int64_t e = (int64_t)blockIdx.y * 256 + threadIdx.x;
+    if (e >= d * d) return;
+    const int s0 = S.row_seg0[r], s1 = S.row_seg0[r + 1];
+    const size_t stride = (size_t)2 * d * d;
+    const bool diag = (e / d) == (e % d);
+    double acc = 0.0;
+    int s = s0;
+    for (; s + 4 <= s1; s += 4) {
+        float g[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) g[q] = aug2[(size_t)(s + q) * stride + e];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float *p = aug2 + (size_t)(s + q) * stride;
+            p[e] = (float)(c * acc);
+            p[d * d + e] = diag ? 1.f : 0.f;
+            acc += (double)g[q];
+        }
+    }
+    for (; s < s1; ++s) {
+        float *p = aug2 + (size_t)s * stride;
+        const float g = p[e];
+        p[e] = (float)(c * acc);
+        p[d * d + e] = diag ? 1.f : 0.f;
+        acc += (double)g;
+    }
+}
+
+// ---------------------------------------------------------------- factor
+template <int D>
+struct FactorCfg {
+    static constexpr int NT = 2 * D;
+    static constexpr int PW = D >= 512 ? 32 : 64;
+};
+
+template <int D>
+__global__ void __launch_bounds__(FactorCfg<D>::NT, 1) factor2_kernel(Segs S, float *aug2) {
+    extern __shared__ float smf[];
+    const int nseg = *S.nseg;
+    for (int s = blockIdx.x; s < nseg; s += gridDim.x) {
+        if (S.k[s] == 0) continue;
+        pc::panel_chol<FactorCfg<D>::PW, FactorCfg<D>::NT>(aug2 + (size_t)s * 2 * D * D, D, 2 * D, D, true,
+                                                           nullptr, true, smf);
+    }
+}
+
+// ---------------------------------------------------------------- A = B B^T
+__device__ __forceinline__ void split3(float v, __nv_bfloat16 &h, __nv_bfloat16 &m, __nv_bfloat16 &l) {
+    h = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(h);
+    m = __float2bfloat16_rn(r1);
+    l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+}
+
+// A_nk = sum_{m >= max(n,k)} B_nm B_km (B upper triangular); 64 x 64 tiles,
+// grid (segment, tile).
+template <int D>
+__global__ void __launch_bounds__(256) ainv_kernel(Segs S, const float *aug2, __nv_bfloat16 *A3) {
+    const int s = blockIdx.x;
+    if (s >= *S.nseg || S.k[s] == 0) return;
+    constexpr int NTL = D / 64;
+    const int I = blockIdx.y / NTL, J = blockIdx.y % NTL;
+    const float *B = aug2 + (size_t)s * 2 * D * D + (size_t)D * D;
+    __shared__ float As[32][65];
+    __shared__ float Bs[32][65];
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    float acc[4][4] = {};
+    const int m_start = (I > J ? I : J) * 64;
+    for (int m0 = m_start; m0 < D; m0 += 32) {
+        for (int e = tid; e < 64 * 32; e += 256) {
+            const int rr = e >> 5, kk = e & 31;
+            As[kk][rr] = B[(size_t)(I * 64 + rr) * D + m0 + kk];
+            Bs[kk][rr] = B[(size_t)(J * 64 + rr) * D + m0 + kk];
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) { a[q] = As[kk][ty * 4 + q]; b[q] = Bs[kk][tx * 4 + q]; }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[q][r] = fmaf(a[q], b[r], acc[q][r]);
+        }
+        __syncthreads();
+    }
+    __nv_bfloat16 *A = A3 + (size_t)s * 3 * D * D;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            __nv_bfloat16 h, m, l;
+            split3(acc[q][r], h, m, l);
+            const size_t o = (size_t)(I * 64 + ty * 4 + q) * D + J * 64 + tx * 4 + r;
+            A[o] = h;
+            A[(size_t)D * D + o] = m;
+            A[(size_t)2 * D * D + o] = l;
+        }
+}
+
+// ---------------------------------------------------------------- tcgen05 K-major GEMM core
+// TMEM[128 x NTOT] (+)= sum over chunks c of A_c (128 x 64) B_c (NTOT x 64)^T.
+// `load(c, a_saddr, b_saddr)` issues the cp.async fills of chunk c (K-major
+// 128-byte swizzle); one thread issues the MMAs; NS stages in flight.
+template <int NTOT, int NS, class Load>
+__device__ __forceinline__ bool tc_gemm_kmajor(uint32_t tbase, int nchunks, uint32_t sbase, uint64_t *mbar,
+                                               Load load, int32_t *st) {
+    constexpr uint32_t A_BYTES = 128 * 128;
+    constexpr uint32_t STAGE = A_BYTES + NTOT * 128;
+    constexpr int NPER = NTOT < 256 ? NTOT : 256;
+    constexpr int NMMA = NTOT / NPER;
+    constexpr uint32_t idesc = tc::idesc_bf16(128, NPER, false, false);
+    bool ok = true;
+    for (int c = 0; c < NS - 1; ++c) {
+        if (c < nchunks) load(c, sbase + (uint32_t)c * STAGE, sbase + (uint32_t)c * STAGE + A_BYTES);
+        tc::cp_async_commit();
+    }
+    for (int c = 0; c < nchunks; ++c) {
+        const int cn = c + NS - 1;
+        if (cn < nchunks) {
+            if (cn >= NS) ok &= tc::mbar_wait(&mbar[cn % NS], (uint32_t)((cn / NS) - 1) & 1u, st);
+            const uint32_t sa = sbase + (uint32_t)(cn % NS) * STAGE;
+            load(cn, sa, sa + A_BYTES);
+        }
+        tc::cp_async_commit();
+        tc::cp_async_wait<NS - 1>();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            tc::fence_after_sync();
+            const uint32_t sa = sbase + (uint32_t)(c % NS) * STAGE, sb = sa + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = tc::sdesc(sa + kk * 32, 16, 1024);
+#pragma unroll
+                for (int nb = 0; nb < NMMA; ++nb) {
+                    const uint64_t bd = tc::sdesc(sb + (uint32_t)nb * 256 * 128 + kk * 32, 16, 1024);
+                    tc::mma_bf16(tbase + (uint32_t)(nb * 256), ad, bd, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                }
+            }
+            tc::mma_commit(&mbar[c % NS]);
+        }
+        __syncthreads();
+    }
+    if (nchunks > 0) ok &= tc::mbar_wait(&mbar[(nchunks - 1) % NS], (uint32_t)((nchunks - 1) / NS) & 1u, st);
+    ok = __syncthreads_and(ok) != 0;
+    tc::fence_after_sync();
+    return ok;
+}
+
+// cp.async fill of a K-major tile: `rows` rows of 64 bf16 from a row-major
+// matrix (row pointer from `rowp(r)`, or zeros when it returns nullptr).
+template <class RowPtr>
+__device__ __forceinline__ void fill_kmajor(uint32_t saddr, int rows, RowPtr rowp) {
+    for (int e = threadIdx.x; e < rows * 8; e += blockDim.x) {
+        const int r = e >> 3, ch = e & 7;
+        const __nv_bfloat16 *g = rowp(r);
+        tc::cp_async16(saddr + tc::kmajor_off(r, ch * 8), g ? (const void *)(g + ch * 8) : (const void *)rowp(-1),
+                       g ? 16u : 0u);
+    }
+}
+
+template <int D>
+struct VCfg {
+    static constexpr int NS = D >= 512 ? 2 : 3;
+    static constexpr uint32_t STAGE = 128 * 128 + D * 128;
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+};
+
+// V = X_s A_s (one 128-position block per CTA), written as three bf16 pieces.
+template <int D>
+__global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+                                                        const __nv_bfloat16 *__restrict__ A3,
+                                                        __nv_bfloat16 *V3, int64_t N, int32_t *st) {
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[VCfg<D>::NS];
+    __shared__ uint32_t tmem_base;
+    const int s = blockIdx.x;
+    if (s >= *S.nseg || S.k[s] == 0) return;
+    const int len = S.len[s];
+    const int mb = blockIdx.y;
+    if (mb * 128 >= len) return;
+    const int64_t start = S.start[s];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, D);
+    if (tid == 0) {
+        for (int i = 0; i < VCfg<D>::NS; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    const __nv_bfloat16 *Xb = H + (start + (int64_t)mb * 128) * D;
+    const int rows_valid = min(128, len - mb * 128);
+    const __nv_bfloat16 *Aseg = A3 + (size_t)s * 3 * D * D;
+    constexpr int KC = D / 64;
+    auto load = [&](int c, uint32_t sa, uint32_t sb) {
+        const int p = c / KC, kc = c % KC;
+        fill_kmajor(sa, 128, [&](int r) -> const __nv_bfloat16 * {
+            return r < 0 ? Xb : (r < rows_valid ? Xb + (int64_t)r * D + kc * 64 : nullptr);
+        });
+        const __nv_bfloat16 *Ap = Aseg + (size_t)p * D * D + kc * 64;
+        fill_kmajor(sb, D, [&](int r) -> const __nv_bfloat16 * { return Ap + (int64_t)(r < 0 ? 0 : r) * D; });
+    };
+    const bool ok = tc_gemm_kmajor<D, VCfg<D>::NS>(tbase, 3 * KC, base, mbar, load, st);
+    if (ok) {
+        const int row = warp * 32 + lane;
+        const bool valid = row < rows_valid;
+        __nv_bfloat16 *v0 = V3 + (size_t)(start + mb * 128 + row) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float v[16];
+            tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            if (valid) {
+                __align__(16) __nv_bfloat16 h[16], m[16], l[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) split3(v[i], h[i], m[i], l[i]);
+                uint4 *d0 = reinterpret_cast<uint4 *>(v0 + c0);
+                uint4 *d1 = reinterpret_cast<uint4 *>(v0 + (size_t)N * D + c0);
+                uint4 *d2 = reinterpret_cast<uint4 *>(v0 + (size_t)2 * N * D + c0);
+                d0[0] = reinterpret_cast<uint4 *>(h)[0]; d0[1] = reinterpret_cast<uint4 *>(h)[1];
+                d1[0] = reinterpret_cast<uint4 *>(m)[0]; d1[1] = reinterpret_cast<uint4 *>(m)[1];
+                d2[0] = reinterpret_cast<uint4 *>(l)[0]; d2[1] = reinterpret_cast<uint4 *>(l)[1];
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, D);
+}
+
+struct KCfg {
+    static constexpr int NS = 4;
+    static constexpr uint32_t STAGE = 128 * 128 + 128 * 128;
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+};
+
+// G'_s = c X_s V^T on the lower 128 x 128 blocks of the segment; grid (segment, 10).
+template <int D>
+__global__ void __launch_bounds__(128, 1) kgemm_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+                                                        const __nv_bfloat16 *__restrict__ V3, int64_t N,
+                                                        float c_rate, float *gp, int32_t *st) {
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[KCfg::NS];
+    __shared__ uint32_t tmem_base;
+    const int s = blockIdx.x;
+    if (s >= *S.nseg || S.k[s] == 0) return;
+    const int t = blockIdx.y;
+    int mi = 0;
+    while ((mi + 1) * (mi + 2) / 2 <= t) ++mi;
+    const int nj = t - mi * (mi + 1) / 2;
+    const int len = S.len[s];
+    if (mi * 128 >= len) return;
+    const int64_t start = S.start[s];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 128);
+    if (tid == 0) {
+        for (int i = 0; i < KCfg::NS; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    const int rows_a = min(128, len - mi * 128), rows_b = min(128, len - nj * 128);
+    const __nv_bfloat16 *Xa = H + (start + (int64_t)mi * 128) * D;
+    const __nv_bfloat16 *Vb = V3 + (size_t)(start + nj * 128) * D;
+    constexpr int KC = D / 64;
+    auto load = [&](int c, uint32_t sa, uint32_t sb) {
+        const int p = c / KC, kc = c % KC;
+        fill_kmajor(sa, 128, [&](int r) -> const __nv_bfloat16 * {
+            return r < 0 ? Xa : (r < rows_a ? Xa + (int64_t)r * D + kc * 64 : nullptr);
+        });
+        const __nv_bfloat16 *Vp = Vb + (size_t)p * N * D;
+        fill_kmajor(sb, 128, [&](int r) -> const __nv_bfloat16 * {
+            return r < 0 ? Vp : (r < rows_b ? Vp + (int64_t)r * D + kc * 64 : nullptr);
+        });
+    };
+    const bool ok = tc_gemm_kmajor<128, KCfg::NS>(tbase, 3 * KC, base, mbar, load, st);
+    if (ok) {
+        const int i = mi * 128 + warp * 32 + lane;
+        const int ld = ldg_of(len);
+        float *G = gp + (size_t)start * kSegMax + (size_t)i * ld + nj * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+            float v[16];
+            tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            if (i < len) {
+                const int j0 = nj * 128 + c0;
+                if (j0 + 16 <= len) {
+                    float4 *dst = reinterpret_cast<float4 *>(G + c0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_float4(c_rate * v[4 * q], c_rate * v[4 * q + 1], c_rate * v[4 * q + 2],
+                                             c_rate * v[4 * q + 3]);
+                } else {
+                    for (int q = 0; q < 16 && j0 + q < len; ++q) G[c0 + q] = c_rate * v[q];
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 128);
+}
+
+// ---------------------------------------------------------------- in-segment Cholesky
+constexpr int kInsegPW = 64, kInsegNT = 512;
+
+__global__ void __launch_bounds__(kInsegNT, 1) inseg_kernel(Segs S, float *gp, float *dR) {
+    extern __shared__ float smi[];
+    const int nseg = *S.nseg;
+    for (int s = blockIdx.x; s < nseg; s += gridDim.x) {
+        if (S.k[s] == 0) continue;
+        const int len = S.len[s];
+        const int64_t start = S.start[s];
+        pc::panel_chol<kInsegPW, kInsegNT>(gp + (size_t)start * kSegMax, ldg_of(len), len, len, false,
+                                           dR + start, false, smi);
+    }
+}
+
+template <int D>
+dbc_status run_tc(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N,
+                  float eps2, float *dR, const Layout2 &L, int32_t *st, cudaStream_t stream) {
+    const double c = (double)D / (double)eps2;
+    const int64_t ns = nseg_upper(rows, N);
+    const int sms = num_sms();
+    seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, L.segs, st);
+    launch_gram_tc<D>(H, ns, L.segs, L.aug2, (size_t)2 * D * D, st, stream);
+    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D + 255) / 256)), 256, 0, stream>>>(L.segs, L.aug2, D, c);
+    using F = FactorCfg<D>;
+    using PF = pc::PanelChol<F::PW, F::NT>;
+    cudaFuncSetAttribute(factor2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PF::SMEM);
+    const int grid_seg = (int)std::min<int64_t>(ns, (int64_t)sms * 8);
+    factor2_kernel<D><<<grid_seg, F::NT, PF::SMEM, stream>>>(L.segs, L.aug2);
+    ainv_kernel<D><<<dim3((unsigned)ns, (unsigned)((D / 64) * (D / 64))), 256, 0, stream>>>(L.segs, L.aug2, L.A3);
+    cudaFuncSetAttribute(vgemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VCfg<D>::SMEM);
+    vgemm_kernel<D><<<dim3((unsigned)ns, 4), 128, VCfg<D>::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, st);
+    cudaFuncSetAttribute(kgemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KCfg::SMEM);
+    kgemm_kernel<D><<<dim3((unsigned)ns, 10), 128, KCfg::SMEM, stream>>>(H, L.segs, L.V3, N, (float)c, L.gp, st);
+    using PI = pc::PanelChol<kInsegPW, kInsegNT>;
+    cudaFuncSetAttribute(inseg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PI::SMEM);
+    inseg_kernel<<<grid_seg, kInsegNT, PI::SMEM, stream>>>(L.segs, L.gp, dR);
+    const size_t smem1 = 64 * 65 * sizeof(double) + (size_t)64 * (D + 1) * sizeof(float);
+    cudaFuncSetAttribute(first_seg_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    first_seg_kernel<__nv_bfloat16><<<(unsigned)std::min<int64_t>(ns, (int64_t)sms * 2), 256, smem1, stream>>>(
+        H, D, L.segs, c, dR);
+    count_launches(10);
+    return launch_status();
+}
+
+}  // namespace cr
+}  // namespace dbc
