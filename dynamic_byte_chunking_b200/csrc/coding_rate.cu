@@ -36,20 +36,29 @@ namespace cr {
 constexpr int PW = 32;          // Cholesky panel width
 constexpr int kSegMax = 512;    // longest segment
 
-__host__ __device__ inline int64_t seg_count(int64_t n) {
+// Segment boundaries of a row: 0, 64, 128, then (lmax = 512) 256 and every
+// multiple of 512, or (lmax = 256) every multiple of 256.  Lengths double
+// until lmax so a segment is never longer than the prefix before it.
+__host__ __device__ inline int seg_k0(int lmax) { return lmax >= 512 ? 4 : 3; }
+
+__host__ __device__ inline int64_t seg_bound(int64_t k, int lmax) {
+    const int k0 = seg_k0(lmax);
+    if (k < k0) return k == 0 ? 0 : (k == 1 ? 64 : (k == 2 ? 128 : 256));
+    return (int64_t)lmax * (k - k0 + 1);
+}
+
+__host__ __device__ inline int64_t seg_count(int64_t n, int lmax) {
     if (n <= 0) return 0;
-    if (n <= 64) return 1;
-    if (n <= 128) return 2;
-    if (n <= 256) return 3;
-    if (n <= 512) return 4;
-    return 4 + (n - 1) / 512;
+    const int k0 = seg_k0(lmax);
+    int64_t c = 0;
+    for (int k = 0; k < k0; ++k) c += seg_bound(k, lmax) < n;
+    if (n > lmax) c += (n - 1) / lmax;
+    return c;
 }
 
-__host__ __device__ inline int64_t seg_bound(int64_t k) {
-    return k == 0 ? 0 : k == 1 ? 64 : k == 2 ? 128 : k == 3 ? 256 : 512 * (k - 3);
+inline int64_t nseg_upper(int64_t rows, int64_t N, int lmax = kSegMax) {
+    return (int64_t)seg_k0(lmax) * rows + N / lmax + 1;
 }
-
-inline int64_t nseg_upper(int64_t rows, int64_t N) { return 4 * rows + N / 512 + 1; }
 
 struct Segs {
     int64_t *start;      // absolute first position
@@ -85,7 +94,7 @@ inline Layout carve(void *ws, int64_t rows, int64_t N, int64_t d) {
 
 // ---------------------------------------------------------------- seg table
 __global__ void __launch_bounds__(1024) seg_table_kernel(const int64_t *offsets, int64_t rows,
-                                                         int64_t T, int64_t N, int64_t ns, Segs S,
+                                                         int64_t T, int64_t N, int64_t ns, int lmax, Segs S,
                                                          int32_t *st) {
     __shared__ int64_t wsum[32];
     __shared__ int64_t carry;
@@ -101,7 +110,7 @@ __global__ void __launch_bounds__(1024) seg_table_kernel(const int64_t *offsets,
                 flag(st, DBC_ERR_BOUNDS);
                 n = 0;
             }
-            cnt = seg_count(n);
+            cnt = seg_count(n, lmax);
         }
         int64_t x = cnt;
         for (int o = 1; o < 32; o <<= 1) {
@@ -123,8 +132,8 @@ __global__ void __launch_bounds__(1024) seg_table_kernel(const int64_t *offsets,
         if (r < rows) {
             S.row_seg0[r] = (int32_t)excl;
             for (int64_t k = 0; k < cnt && excl + k < ns; ++k) {
-                const int64_t s0 = seg_bound(k);
-                const int64_t s1 = min(n, seg_bound(k + 1));
+                const int64_t s0 = seg_bound(k, lmax);
+                const int64_t s1 = min(n, seg_bound(k + 1, lmax));
                 const int64_t s = excl + k;
                 S.start[s] = a + s0;
                 S.len[s] = (int32_t)(s1 - s0);
@@ -579,7 +588,7 @@ dbc_status run(const IN *H, const int64_t *offsets, int64_t rows, int64_t T, int
     const double c = (double)d / (double)eps2;
     const int64_t ns = nseg_upper(rows, N);
     const int sms = num_sms();
-    seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, L.segs, st);
+    seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kSegMax, L.segs, st);
     launch_gram(H, d, ns, L, st, stream);
     prefix_kernel<<<dim3((unsigned)rows, (unsigned)((d * d + 255) / 256)), 256, 0, stream>>>(
         L.segs, L.aug, d, c);
@@ -615,7 +624,8 @@ extern "C" size_t chunk_coding_rate_workspace(int64_t rows, int64_t T, int64_t N
     (void)T;
     if (rows < 0 || N < 0 || d <= 0) return 0;
     // large enough for either path (the dtype is not an argument of the query)
-    return std::max(cr::carve(nullptr, rows, N, d).bytes, cr::carve2(nullptr, rows, N, d).bytes);
+    return std::max({cr::carve(nullptr, rows, N, d).bytes, cr::carve2(nullptr, rows, N, d).bytes,
+                     cr::carve3(nullptr, rows, N, d).bytes});
 }
 
 extern "C" dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t *offsets,
@@ -628,8 +638,15 @@ extern "C" dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t 
     if (!offsets && N != rows * T) return DBC_ERR_INVALID_ARG;
     if (N == 0 || rows == 0) return DBC_OK;
     if (!H || !dR || !aligned16(H)) return DBC_ERR_INVALID_ARG;
-    if (cr::nseg_upper(rows, N) > INT32_MAX / 2) return DBC_ERR_UNSUPPORTED;
+    if (cr::nseg_upper(rows, N, 256) > INT32_MAX / 2) return DBC_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == DBC_BF16 && d == 256) {
+        const cr::Layout3 need3 = cr::carve3(nullptr, rows, N, d);
+        if (!ws || ws_bytes < need3.bytes || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)))
+            return DBC_ERR_WORKSPACE;
+        return cr::run_tmem(static_cast<const __nv_bfloat16 *>(H), offsets, rows, T, N, eps2, dR,
+                            cr::carve3(ws, rows, N, d), dev_status, s);
+    }
     if (use_tensor_path(dtype, d)) {
         const cr::Layout2 need2 = cr::carve2(nullptr, rows, N, d);
         if (!ws || ws_bytes < need2.bytes || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)))

@@ -12,6 +12,7 @@
 //   kgemm:  G'_s = c X_s V^T on tcgen05 (three passes), lower 128-blocks;
 //   inseg:  panel Cholesky of I + G'_s with the identity implicit; the
 //           excess e_t of each diagonal gives dR_t = log1p(e_t) / 2.
+// A row's first segment takes the same path with P = 0 (so A = I).
 // G'_s = c X_s M_s^{-1} X_s^T is the in-segment Gram in the frame whitened
 // by the segment's start state, so its Cholesky diagonal is the per-position
 // Schur complement 1 + c h_t^T M_{t-1}^{-1} h_t (matrix determinant lemma).
@@ -54,14 +55,12 @@ inline Layout2 carve2(void *ws, int64_t rows, int64_t N, int64_t d) {
 
 // ---------------------------------------------------------------- prefix
 // In place over a row's segments: Gram -> P_s = c sum_{s'<s} G_s' (float64
-// running sum, fp32 store); the appended block of each matrix becomes I.
-__global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c) {
+// running sum, fp32 store).
+__global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c, size_t stride) {
     const int64_t r = blockIdx.x;
     const int64_t e = (int64_t)blockIdx.y * 256 + threadIdx.x;
     if (e >= d * d) return;
     const int s0 = S.row_seg0[r], s1 = S.row_seg0[r + 1];
-    const size_t stride = (size_t)2 * d * d;
-    const bool diag = (e / d) == (e % d);
     double acc = 0.0;
     int s = s0;
     for (; s + 4 <= s1; s += 4) {
@@ -70,9 +69,7 @@ __global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64
         for (int q = 0; q < 4; ++q) g[q] = aug2[(size_t)(s + q) * stride + e];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            float *p = aug2 + (size_t)(s + q) * stride;
-            p[e] = (float)(c * acc);
-            p[d * d + e] = diag ? 1.f : 0.f;
+            aug2[(size_t)(s + q) * stride + e] = (float)(c * acc);
             acc += (double)g[q];
         }
     }
@@ -80,7 +77,6 @@ __global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64
         float *p = aug2 + (size_t)s * stride;
         const float g = p[e];
         p[e] = (float)(c * acc);
-        p[d * d + e] = diag ? 1.f : 0.f;
         acc += (double)g;
     }
 }
@@ -97,9 +93,14 @@ __global__ void __launch_bounds__(FactorCfg<D>::NT, 1) factor2_kernel(Segs S, fl
     extern __shared__ float smf[];
     const int nseg = *S.nseg;
     for (int s = blockIdx.x; s < nseg; s += gridDim.x) {
-        if (S.k[s] == 0) continue;
-        pc::panel_chol<FactorCfg<D>::PW, FactorCfg<D>::NT>(aug2 + (size_t)s * 2 * D * D, D, 2 * D, D, true,
-                                                           nullptr, true, smf);
+        float *Ms = aug2 + (size_t)s * 2 * D * D;
+        float4 *bot = reinterpret_cast<float4 *>(Ms + (size_t)D * D);     // appended block <- I
+        for (int e = threadIdx.x; e < D * D / 4; e += FactorCfg<D>::NT) {
+            const int i = (4 * e) / D, j = (4 * e) % D;
+            bot[e] = make_float4(i == j, i == j + 1, i == j + 2, i == j + 3);
+        }
+        __syncthreads();
+        pc::panel_chol<FactorCfg<D>::PW, FactorCfg<D>::NT>(Ms, D, 2 * D, D, true, nullptr, true, smf);
     }
 }
 
@@ -116,7 +117,7 @@ __device__ __forceinline__ void split3(float v, __nv_bfloat16 &h, __nv_bfloat16 
 template <int D>
 __global__ void __launch_bounds__(256) ainv_kernel(Segs S, const float *aug2, __nv_bfloat16 *A3) {
     const int s = blockIdx.x;
-    if (s >= *S.nseg || S.k[s] == 0) return;
+    if (s >= *S.nseg) return;
     constexpr int NTL = D / 64;
     const int I = blockIdx.y / NTL, J = blockIdx.y % NTL;
     const float *B = aug2 + (size_t)s * 2 * D * D + (size_t)D * D;
@@ -231,12 +232,12 @@ struct VCfg {
 template <int D>
 __global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
                                                         const __nv_bfloat16 *__restrict__ A3,
-                                                        __nv_bfloat16 *V3, int64_t N, int32_t *st) {
+                                                        __nv_bfloat16 *V3, int64_t N, float scale, int32_t *st) {
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[VCfg<D>::NS];
     __shared__ uint32_t tmem_base;
     const int s = blockIdx.x;
-    if (s >= *S.nseg || S.k[s] == 0) return;
+    if (s >= *S.nseg) return;
     const int len = S.len[s];
     const int mb = blockIdx.y;
     if (mb * 128 >= len) return;
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__re
             if (valid) {
                 __align__(16) __nv_bfloat16 h[16], m[16], l[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) split3(v[i], h[i], m[i], l[i]);
+                for (int i = 0; i < 16; ++i) split3(scale * v[i], h[i], m[i], l[i]);
                 uint4 *d0 = reinterpret_cast<uint4 *>(v0 + c0);
                 uint4 *d1 = reinterpret_cast<uint4 *>(v0 + (size_t)N * D + c0);
                 uint4 *d2 = reinterpret_cast<uint4 *>(v0 + (size_t)2 * N * D + c0);
@@ -306,7 +307,7 @@ __global__ void __launch_bounds__(128, 1) kgemm_kernel(const __nv_bfloat16 *__re
     __shared__ uint64_t mbar[KCfg::NS];
     __shared__ uint32_t tmem_base;
     const int s = blockIdx.x;
-    if (s >= *S.nseg || S.k[s] == 0) return;
+    if (s >= *S.nseg) return;
     const int t = blockIdx.y;
     int mi = 0;
     while ((mi + 1) * (mi + 2) / 2 <= t) ++mi;
@@ -374,7 +375,6 @@ __global__ void __launch_bounds__(kInsegNT, 1) inseg_kernel(Segs S, float *gp, f
     extern __shared__ float smi[];
     const int nseg = *S.nseg;
     for (int s = blockIdx.x; s < nseg; s += gridDim.x) {
-        if (S.k[s] == 0) continue;
         const int len = S.len[s];
         const int64_t start = S.start[s];
         pc::panel_chol<kInsegPW, kInsegNT>(gp + (size_t)start * kSegMax, ldg_of(len), len, len, false,
@@ -388,9 +388,10 @@ dbc_status run_tc(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, 
     const double c = (double)D / (double)eps2;
     const int64_t ns = nseg_upper(rows, N);
     const int sms = num_sms();
-    seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, L.segs, st);
+    seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kSegMax, L.segs, st);
     launch_gram_tc<D>(H, ns, L.segs, L.aug2, (size_t)2 * D * D, st, stream);
-    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D + 255) / 256)), 256, 0, stream>>>(L.segs, L.aug2, D, c);
+    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D + 255) / 256)), 256, 0, stream>>>(L.segs, L.aug2, D, c,
+                                                                                            (size_t)2 * D * D);
     using F = FactorCfg<D>;
     using PF = pc::PanelChol<F::PW, F::NT>;
     cudaFuncSetAttribute(factor2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PF::SMEM);
@@ -398,17 +399,77 @@ dbc_status run_tc(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, 
     factor2_kernel<D><<<grid_seg, F::NT, PF::SMEM, stream>>>(L.segs, L.aug2);
     ainv_kernel<D><<<dim3((unsigned)ns, (unsigned)((D / 64) * (D / 64))), 256, 0, stream>>>(L.segs, L.aug2, L.A3);
     cudaFuncSetAttribute(vgemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VCfg<D>::SMEM);
-    vgemm_kernel<D><<<dim3((unsigned)ns, 4), 128, VCfg<D>::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, st);
+    vgemm_kernel<D><<<dim3((unsigned)ns, 4), 128, VCfg<D>::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, 1.f, st);
     cudaFuncSetAttribute(kgemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KCfg::SMEM);
     kgemm_kernel<D><<<dim3((unsigned)ns, 10), 128, KCfg::SMEM, stream>>>(H, L.segs, L.V3, N, (float)c, L.gp, st);
     using PI = pc::PanelChol<kInsegPW, kInsegNT>;
     cudaFuncSetAttribute(inseg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PI::SMEM);
     inseg_kernel<<<grid_seg, kInsegNT, PI::SMEM, stream>>>(L.segs, L.gp, dR);
-    const size_t smem1 = 64 * 65 * sizeof(double) + (size_t)64 * (D + 1) * sizeof(float);
-    cudaFuncSetAttribute(first_seg_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-    first_seg_kernel<__nv_bfloat16><<<(unsigned)std::min<int64_t>(ns, (int64_t)sms * 2), 256, smem1, stream>>>(
-        H, D, L.segs, c, dR);
-    count_launches(10);
+    count_launches(9);
+    return launch_status();
+}
+
+// ================================================================ d = 256: TMEM-resident factorizations
+// Segments of at most 256 positions: the start state's factorization and
+// inverse (FACTOR) and the in-segment Cholesky (INSEG) each run inside one
+// SM's tensor memory.
+constexpr int kLmaxTmem = 256;
+
+struct Layout3 {
+    Segs segs;
+    float *P;               // per segment: [D][D] Gram -> c-scaled prefix
+    __nv_bfloat16 *Bscr;    // per segment: [3][D][D] pieces of L^{-T}
+    __nv_bfloat16 *A3;      // per segment: [3][D][D] pieces of M_s^{-1}
+    __nv_bfloat16 *V3;      // [3][N][D] pieces of c X_s M_s^{-1}
+    size_t bytes;
+};
+
+inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d) {
+    Carver c(ws);
+    const int64_t ns = nseg_upper(rows, N, kLmaxTmem);
+    Layout3 L;
+    L.segs.start = c.take<int64_t>(ns);
+    L.segs.len = c.take<int32_t>(ns);
+    L.segs.row = c.take<int32_t>(ns);
+    L.segs.k = c.take<int32_t>(ns);
+    L.segs.row_seg0 = c.take<int32_t>(rows + 1);
+    L.segs.nseg = c.take<int32_t>(1);
+    L.P = c.take<float>((size_t)ns * d * d);
+    L.Bscr = c.take<__nv_bfloat16>((size_t)ns * 3 * d * d);
+    L.A3 = c.take<__nv_bfloat16>((size_t)ns * 3 * d * d);
+    L.V3 = c.take<__nv_bfloat16>((size_t)3 * N * d + 8);
+    L.bytes = c.off;
+    return L;
+}
+
+}  // namespace cr
+}  // namespace dbc
+
+#include "tmem_chol.cuh"
+
+namespace dbc {
+namespace cr {
+
+inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N,
+                           float eps2, float *dR, const Layout3 &L, int32_t *st, cudaStream_t stream) {
+    constexpr int D = 256;
+    const double c = (double)D / (double)eps2;
+    const int64_t ns = nseg_upper(rows, N, kLmaxTmem);
+    const int sms = num_sms();
+    seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kLmaxTmem, L.segs, st);
+    launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
+    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D + 255) / 256)), 256, 0, stream>>>(L.segs, L.P, D, c,
+                                                                                            (size_t)D * D);
+    const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
+    cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
+    cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(H, L.segs, L.P, L.Bscr, L.A3, nullptr, N,
+                                                                         dR, st);
+    cudaFuncSetAttribute(vgemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VCfg<D>::SMEM);
+    vgemm_kernel<D><<<dim3((unsigned)ns, 2), 128, VCfg<D>::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, (float)c, st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(H, L.segs, nullptr, nullptr, nullptr,
+                                                                          L.V3, N, dR, st);
+    count_launches(6);
     return launch_status();
 }
 

@@ -1,0 +1,412 @@
+// Blocked Cholesky of (I + S) held entirely in tensor memory (d = 256).
+//
+// A 256 x 256 fp32 matrix fills one SM's TMEM: rows 0..127 sit in lanes
+// 0..127 at columns [0, 256), rows 128..255 in the same lanes at columns
+// [256, 512).  256 threads: thread (warp w, lane l) owns row
+// (w/4)*128 + (w%4)*32 + l, the lanes its warp may address.  The identity is
+// implicit: the stored diagonal is the excess e, the factor's diagonal is
+// sqrt(1 + e).
+//
+// Per 64-column panel: every thread loads its row's 64 panel entries with
+// tcgen05.ld, the panel is factored in registers (two barriers per column),
+// the panel rows are split into three bf16 pieces (hi + mid + lo carries the
+// fp32 value) and staged in shared memory, and the trailing columns are
+// updated in place by tcgen05 MMAs with negated A over the six piece
+// products whose sum is accurate to fp32 (hi.hi, hi.mid, mid.hi, hi.lo,
+// lo.hi, mid.mid).  Two uses:
+//
+//  * FACTOR (segment start state M_s = I + P_s): the upper triangle, which
+//    starts at zero, carries B = L^{-T} along (row i of the identity solved
+//    against the factor, B_ii = 1 / L_ii), so one sweep yields both; the
+//    panels of B are saved and A = B B^T = M_s^{-1} is formed at the end on
+//    tcgen05 and stored as three bf16 pieces.
+//  * INSEG (one segment): G' = X (c V)^T is accumulated straight into TMEM
+//    (V = X_s A_s in pieces), factored in place, and the excess of each
+//    column gives dR_t = log1p(e_t) / 2.
+#pragma once
+
+#include "tc.cuh"
+
+namespace dbc {
+namespace cr {
+
+struct TmemChol {
+    static constexpr int NT = 256;
+    static constexpr uint32_t XT = 128 * 128;             // 128-row x 64-K bf16 tile
+    static constexpr uint32_t PIECE = 256 * 128;          // 256-row x 64-K bf16 tile
+    static constexpr uint32_t PANEL = 3 * PIECE;          // staged panel (three pieces)
+    static constexpr uint32_t GSTAGE = 2 * XT + PIECE;    // G' GEMM stage: X (two row blocks) + V piece
+    static constexpr uint32_t REGION = (2 * GSTAGE > PANEL) ? 2 * GSTAGE : PANEL;
+    static constexpr size_t SMEM = REGION + 1024;
+};
+
+// Six piece products of a three-way split (dropped terms are below 2^-24):
+// hi.hi, hi.mid, mid.hi, hi.lo, lo.hi, mid.mid.
+__device__ __forceinline__ constexpr int pair_a(int i) { return i == 2 ? 1 : (i == 4 ? 2 : (i == 5 ? 1 : 0)); }
+__device__ __forceinline__ constexpr int pair_b(int i) { return i == 1 ? 1 : (i == 3 ? 2 : (i == 5 ? 1 : 0)); }
+
+__device__ __forceinline__ void split3v(float v, uint16_t &h, uint16_t &m, uint16_t &l) {
+    const __nv_bfloat16 bh = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(bh);
+    const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 bl = __float2bfloat16_rn(r1 - __bfloat162float(bm));
+    h = __bfloat16_as_ushort(bh);
+    m = __bfloat16_as_ushort(bm);
+    l = __bfloat16_as_ushort(bl);
+}
+
+// Stages 64 values of one row as three K-major pieces (row `row` of each
+// 256-row tile) and, when gdst != nullptr, also writes them to global
+// pieces gdst[p * pstride + k] (row-major bf16).
+__device__ __forceinline__ void stage_row(uint32_t region, int row, const float (&a)[64], __nv_bfloat16 *gdst,
+                                          size_t pstride) {
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {
+        uint32_t hh[4], mm[4], ll[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint16_t h0, m0, l0, h1, m1, l1;
+            split3v(a[k8 * 8 + 2 * q], h0, m0, l0);
+            split3v(a[k8 * 8 + 2 * q + 1], h1, m1, l1);
+            hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
+            ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+        }
+        const uint32_t off = tc::kmajor_off(row, k8 * 8);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + off), "r"(hh[0]), "r"(hh[1]),
+                     "r"(hh[2]), "r"(hh[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + TmemChol::PIECE + off), "r"(mm[0]),
+                     "r"(mm[1]), "r"(mm[2]), "r"(mm[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + 2 * TmemChol::PIECE + off),
+                     "r"(ll[0]), "r"(ll[1]), "r"(ll[2]), "r"(ll[3])
+                     : "memory");
+        if (gdst) {
+            *reinterpret_cast<uint4 *>(gdst + k8 * 8) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+            *reinterpret_cast<uint4 *>(gdst + pstride + k8 * 8) = make_uint4(mm[0], mm[1], mm[2], mm[3]);
+            *reinterpret_cast<uint4 *>(gdst + 2 * pstride + k8 * 8) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
+        }
+    }
+}
+
+// D[block b rows, columns c0 .. c0+N) (+/-)= sum of the six piece products of
+// A (rows a_row0 .. +128 of the staged tiles) and B (rows b_row0 .. +N).
+__device__ __forceinline__ void issue_split_mma(uint32_t d_tmem, uint32_t region_a, uint32_t region_b,
+                                                int a_row0, int b_row0, uint32_t idesc, bool first) {
+#pragma unroll
+    for (int pr = 0; pr < 6; ++pr) {
+        const uint32_t pa = region_a + (uint32_t)pair_a(pr) * TmemChol::PIECE + (uint32_t)a_row0 * 128;
+        const uint32_t pb = region_b + (uint32_t)pair_b(pr) * TmemChol::PIECE + (uint32_t)b_row0 * 128;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(d_tmem, tc::sdesc(pa + kk * 32, 16, 1024), tc::sdesc(pb + kk * 32, 16, 1024), idesc,
+                         (first && pr == 0 && kk == 0) ? 0u : 1u);
+    }
+}
+
+// Runtime N of the negated trailing update (N = 256 - j1, a multiple of 64).
+__device__ __forceinline__ uint32_t idesc_neg(int N) { return tc::idesc_bf16(128, N, false, false, true); }
+
+template <bool FACTOR>
+__global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
+    const __nv_bfloat16 *__restrict__ H, Segs S, const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr,
+    __nv_bfloat16 *A3, const __nv_bfloat16 *__restrict__ V3, int64_t N, float *dR, int32_t *st) {
+    constexpr int D = 256;
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ float s_col[64];
+    __shared__ float s_e;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int blk = warp >> 2, lb = (warp & 3) * 32;
+    const int row = blk * 128 + lb + lane;
+    const uint32_t region = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
+    if (tid == 0) {
+        tc::mbar_init(&mbar[0], 1);
+        tc::mbar_init(&mbar[1], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    const uint32_t trow = tbase + ((uint32_t)lb << 16) + (uint32_t)(blk * 256);
+    uint32_t ph0 = 0, ph1 = 0;      // mbarrier phases (uniform across threads)
+    bool ok = true;
+    const int nseg = *S.nseg;
+
+    for (int s = blockIdx.x; s < nseg && ok; s += gridDim.x) {
+        const int len = S.len[s];
+        const int64_t start = S.start[s];
+        const int n = FACTOR ? D : len;
+
+        // ---------------- load the matrix into TMEM
+        if (FACTOR) {
+            const float *P = Pbuf + (size_t)s * D * D;            // c-scaled prefix Gram
+            float *stg = reinterpret_cast<float *>(smraw + (region - tc::smem_u32(smraw)));
+            for (int q = 0; q < D / 64; ++q) {
+                for (int e = tid; e < D * 16; e += TmemChol::NT) {           // 256 rows x 16 float4
+                    const int r = e >> 4, c4 = e & 15;
+                    const float4 x = *reinterpret_cast<const float4 *>(P + (size_t)r * D + q * 64 + c4 * 4);
+                    float *d = stg + r * 65 + c4 * 4;
+                    d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = q * 64 + j * 16 + i;
+                        v[i] = col <= row ? stg[row * 65 + j * 16 + i] : 0.f;
+                    }
+                    tc::tmem_st16(trow + (uint32_t)(q * 64 + j * 16), v);
+                }
+                __syncthreads();
+            }
+            tc::tmem_wait_st();
+        } else {
+            // G' = X (c V)^T over 3 pieces x (D/64) feature chunks, two stages
+            const __nv_bfloat16 *X = H + start * D;
+            constexpr int KC = D / 64, NCH = 3 * KC;
+            auto load = [&](int c, uint32_t sb) {
+                const int p = c / KC, kc = c % KC;
+                for (int e = tid; e < 256 * 8; e += TmemChol::NT) {
+                    const int r = e >> 3, ch = e & 7;
+                    const bool in = r < len;
+                    const __nv_bfloat16 *gx = X + (size_t)(in ? r : 0) * D + kc * 64 + ch * 8;
+                    const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : TmemChol::XT + tc::kmajor_off(r - 128, ch * 8);
+                    tc::cp_async16(sb + xo, gx, in ? 16u : 0u);
+                    const __nv_bfloat16 *gv = V3 + (size_t)p * N * D + (size_t)(start + (in ? r : 0)) * D + kc * 64 + ch * 8;
+                    tc::cp_async16(sb + 2 * TmemChol::XT + tc::kmajor_off(r, ch * 8), gv, in ? 16u : 0u);
+                }
+            };
+            constexpr uint32_t idg = tc::idesc_bf16(128, 256, false, false);
+            load(0, region);
+            tc::cp_async_commit();
+            for (int c = 0; c < NCH; ++c) {
+                if (c + 1 < NCH) {
+                    if (c >= 1) {     // stage (c+1)%2 was read by the MMAs of chunk c-1
+                        ok &= tc::mbar_wait(&mbar[(c + 1) & 1], ((c + 1) & 1) ? ph1 : ph0, st);
+                        if ((c + 1) & 1) ph1 ^= 1; else ph0 ^= 1;
+                    }
+                    load(c + 1, region + (uint32_t)((c + 1) & 1) * TmemChol::GSTAGE);
+                }
+                tc::cp_async_commit();
+                tc::cp_async_wait<1>();
+                tc::fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tc::fence_after_sync();
+                    const uint32_t sb = region + (uint32_t)(c & 1) * TmemChol::GSTAGE;
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_bf16(tbase + (uint32_t)(b * 256), tc::sdesc(sb + b * TmemChol::XT + kk * 32, 16, 1024),
+                                         tc::sdesc(sb + 2 * TmemChol::XT + kk * 32, 16, 1024), idg,
+                                         (c > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&mbar[c & 1]);
+                }
+                __syncthreads();
+            }
+            // wait for the last two chunks' MMAs
+            for (int c = (NCH >= 2 ? NCH - 2 : 0); c < NCH; ++c) {
+                ok &= tc::mbar_wait(&mbar[c & 1], (c & 1) ? ph1 : ph0, st);
+                if (c & 1) ph1 ^= 1; else ph0 ^= 1;
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+
+        // ---------------- panels
+        __nv_bfloat16 *Bs = FACTOR ? Bscr + (size_t)s * 3 * D * D : nullptr;
+        for (int j0 = 0; j0 < n; j0 += 64) {
+            const int nb = min(64, n - j0);
+            const int j1 = j0 + nb;
+            float v[64];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float t16[16];
+                tc::tmem_ld16(trow + (uint32_t)(j0 + j * 16), t16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[j * 16 + i] = t16[i];
+            }
+            if (FACTOR && row >= j0 && row < j1) {
+                // this row's B entries right of its diagonal start from zero: B_im = 0 for m < i,
+                // so nothing before this panel contributes to them
+#pragma unroll
+                for (int k = 0; k < 64; ++k)
+                    if (j0 + k > row) v[k] = 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < 64; ++k) {
+                if (k < nb) {
+                    const int kk = j0 + k;
+                    if (row == kk) s_e = v[k];
+                    __syncthreads();
+                    const float e = s_e;
+                    const float l = sqrtf(1.f + e);
+                    float a;
+                    if (row == kk) {
+                        v[k] = l;
+                        a = 1.f / l;
+                        if (!FACTOR) dR[start + kk] = 0.5f * log1pf(e);
+                    } else {
+                        v[k] = v[k] / l;
+                        a = v[k];
+                    }
+                    if (row > kk && row < j0 + 64) s_col[row - j0] = v[k];
+                    __syncthreads();
+                    if (!FACTOR) {
+                        if (row > kk) {
+#pragma unroll
+                            for (int p = k + 1; p < 64; ++p) v[p] = fmaf(-a, s_col[p], v[p]);
+                        }
+                    } else if (row > kk) {
+                        // L role: only this row's lower part (its upper part holds B, and B_i,kk = 0)
+#pragma unroll
+                        for (int p = k + 1; p < 64; ++p)
+                            if (j0 + p <= row) v[p] = fmaf(-a, s_col[p], v[p]);
+                    } else {
+                        // B role (row <= kk): B_i,p -= B_i,kk L_p,kk, with B_ii = 1 / L_ii
+#pragma unroll
+                        for (int p = k + 1; p < 64; ++p) v[p] = fmaf(-a, s_col[p], v[p]);
+                    }
+                }
+            }
+            // operand rows: FACTOR rows < j1 carry B (0 below the diagonal, 1/L_ii on it),
+            // INSEG rows < j1 are not updated (zero); rows >= j1 carry L.
+            if (row < j1) {
+#pragma unroll
+                for (int k = 0; k < 64; ++k) {
+                    const int col = j0 + k;
+                    v[k] = !FACTOR ? 0.f : (col < row ? 0.f : (col == row ? 1.f / v[k] : v[k]));
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 64; ++k)
+                    if (k >= nb) v[k] = 0.f;
+            }
+            if (FACTOR) {
+                // B panel (rows >= j1 are zero there) -> global; operand rows -> smem
+                __nv_bfloat16 *g = Bs + (size_t)row * D + j0;
+                if (row < j1) {
+                    stage_row(region, row, v, g, (size_t)D * D);
+                } else {
+                    stage_row(region, row, v, nullptr, 0);
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int p = 0; p < 3; ++p)
+#pragma unroll
+                        for (int k8 = 0; k8 < 8; ++k8) *reinterpret_cast<uint4 *>(g + (size_t)p * D * D + k8 * 8) = z;
+                }
+            } else if (j1 < n) {
+                stage_row(region, row, v, nullptr, 0);
+            }
+            if (FACTOR && j1 < n && row >= j0 && row < j1) {
+                // the trailing updates of earlier panels reached this row's upper part while it was an
+                // L row; its B entries right of the panel start from zero (warps of the diagonal block)
+                float z[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) z[i] = 0.f;
+                for (int c0 = j1; c0 < D; c0 += 16) tc::tmem_st16(trow + (uint32_t)c0, z);
+                tc::tmem_wait_st();
+            }
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            __syncthreads();
+            if (j1 < n) {
+                if (tid == 0) {
+                    tc::fence_after_sync();
+                    const uint32_t idn = idesc_neg(256 - j1);
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        if (!FACTOR && (b + 1) * 128 <= j1) continue;
+                        issue_split_mma(tbase + (uint32_t)(b * 256 + j1), region, region, b * 128, j1, idn, false);
+                    }
+                    tc::mma_commit(&mbar[0]);
+                }
+                ok &= tc::mbar_wait(&mbar[0], ph0, st);
+                ph0 ^= 1;
+                tc::fence_after_sync();
+                ok = __syncthreads_and(ok) != 0;
+                if (!ok) break;
+            } else {
+                tc::fence_before_sync();
+                __syncthreads();
+                tc::fence_after_sync();
+            }
+        }
+        if (!ok) break;
+
+        // ---------------- FACTOR: A = B B^T from the saved panels, split into pieces
+        if (FACTOR) {
+            for (int q = 0; q < D / 64; ++q) {
+                for (int e = tid; e < 3 * 256 * 8; e += TmemChol::NT) {
+                    const int p = e / 2048, r = (e >> 3) & 255, ch = e & 7;
+                    const bool nz = r < q * 64 + 64;        // B rows beyond are zero in these columns
+                    const __nv_bfloat16 *gsrc = Bs + (size_t)p * D * D + (size_t)(nz ? r : 0) * D + q * 64 + ch * 8;
+                    tc::cp_async16(region + (uint32_t)p * TmemChol::PIECE + tc::kmajor_off(r, ch * 8), gsrc,
+                                   nz ? 16u : 0u);
+                }
+                tc::cp_async_commit();
+                tc::cp_async_wait<0>();
+                tc::fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tc::fence_after_sync();
+                    constexpr uint32_t idp = tc::idesc_bf16(128, 256, false, false);
+                    for (int b = 0; b < 2; ++b) {
+                        if (b == 1 && q < 2) continue;          // rows 128.. of B vanish in columns < 128
+                        issue_split_mma(tbase + (uint32_t)(b * 256), region, region, b * 128, 0, idp,
+                                        b == 0 ? (q == 0) : (q == 2));
+                    }
+                    tc::mma_commit(&mbar[0]);
+                }
+                ok &= tc::mbar_wait(&mbar[0], ph0, st);
+                ph0 ^= 1;
+                tc::fence_after_sync();
+                ok = __syncthreads_and(ok) != 0;
+                if (!ok) break;
+            }
+            if (!ok) break;
+            __nv_bfloat16 *A = A3 + (size_t)s * 3 * D * D + (size_t)row * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float t16[16];
+                tc::tmem_ld16(trow + (uint32_t)c0, t16);
+                uint32_t hh[8], mm[8], ll[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    uint16_t h0, m0, l0, h1, m1, l1;
+                    split3v(t16[2 * q], h0, m0, l0);
+                    split3v(t16[2 * q + 1], h1, m1, l1);
+                    hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                    mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
+                    ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                }
+                uint4 *d0 = reinterpret_cast<uint4 *>(A + c0);
+                uint4 *d1 = reinterpret_cast<uint4 *>(A + (size_t)D * D + c0);
+                uint4 *d2 = reinterpret_cast<uint4 *>(A + (size_t)2 * D * D + c0);
+                d0[0] = make_uint4(hh[0], hh[1], hh[2], hh[3]); d0[1] = make_uint4(hh[4], hh[5], hh[6], hh[7]);
+                d1[0] = make_uint4(mm[0], mm[1], mm[2], mm[3]); d1[1] = make_uint4(mm[4], mm[5], mm[6], mm[7]);
+                d2[0] = make_uint4(ll[0], ll[1], ll[2], ll[3]); d2[1] = make_uint4(ll[4], ll[5], ll[6], ll[7]);
+            }
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 512);
+}
+
+}  // namespace cr
+}  // namespace dbc
