@@ -58,26 +58,27 @@ inline Layout2 carve2(void *ws, int64_t rows, int64_t N, int64_t d) {
 // running sum, fp32 store).
 __global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c, size_t stride) {
     const int64_t r = blockIdx.x;
-    const int64_t e = (int64_t)blockIdx.y * 256 + threadIdx.x;
-    if (e >= d * d) return;
+    const int64_t e4 = (int64_t)blockIdx.y * 256 + threadIdx.x;        // float4 index
+    if (e4 * 4 >= d * d) return;
     const int s0 = S.row_seg0[r], s1 = S.row_seg0[r + 1];
-    double acc = 0.0;
-    int s = s0;
-    for (; s + 4 <= s1; s += 4) {
-        float g[4];
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int sb = s0; sb < s1; sb += 16) {
+        const int cnt = min(16, s1 - sb);
+        float4 g[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) g[q] = aug2[(size_t)(s + q) * stride + e];
+        for (int q = 0; q < 16; ++q)                 // all loads in flight before the running sum
+            if (q < cnt) g[q] = *reinterpret_cast<const float4 *>(aug2 + (size_t)(sb + q) * stride + 4 * e4);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            aug2[(size_t)(s + q) * stride + e] = (float)(c * acc);
-            acc += (double)g[q];
+        for (int q = 0; q < 16; ++q) {
+            if (q < cnt) {
+                *reinterpret_cast<float4 *>(aug2 + (size_t)(sb + q) * stride + 4 * e4) =
+                    make_float4((float)(c * acc[0]), (float)(c * acc[1]), (float)(c * acc[2]), (float)(c * acc[3]));
+                acc[0] += (double)g[q].x;
+                acc[1] += (double)g[q].y;
+                acc[2] += (double)g[q].z;
+                acc[3] += (double)g[q].w;
+            }
         }
-    }
-    for (; s < s1; ++s) {
-        float *p = aug2 + (size_t)s * stride;
-        const float g = p[e];
-        p[e] = (float)(c * acc);
-        acc += (double)g;
     }
 }
 
@@ -390,8 +391,8 @@ dbc_status run_tc(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, 
     const int sms = num_sms();
     seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kSegMax, L.segs, st);
     launch_gram_tc<D>(H, ns, L.segs, L.aug2, (size_t)2 * D * D, st, stream);
-    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D + 255) / 256)), 256, 0, stream>>>(L.segs, L.aug2, D, c,
-                                                                                            (size_t)2 * D * D);
+    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
+        L.segs, L.aug2, D, c, (size_t)2 * D * D);
     using F = FactorCfg<D>;
     using PF = pc::PanelChol<F::PW, F::NT>;
     cudaFuncSetAttribute(factor2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PF::SMEM);
@@ -458,8 +459,8 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     const int sms = num_sms();
     seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kLmaxTmem, L.segs, st);
     launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
-    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D + 255) / 256)), 256, 0, stream>>>(L.segs, L.P, D, c,
-                                                                                            (size_t)D * D);
+    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
+        L.segs, L.P, D, c, (size_t)D * D);
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);

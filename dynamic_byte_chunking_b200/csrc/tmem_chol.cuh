@@ -37,8 +37,41 @@ struct TmemChol {
     static constexpr uint32_t PANEL = 3 * PIECE;          // staged panel (three pieces)
     static constexpr uint32_t GSTAGE = 2 * XT + PIECE;    // G' GEMM stage: X (two row blocks) + V piece
     static constexpr uint32_t REGION = (2 * GSTAGE > PANEL) ? 2 * GSTAGE : PANEL;
-    static constexpr size_t SMEM = REGION + 1024;
+    static constexpr uint32_t DONE = 256 * 65 * 4;           // finished panel values [256][65] fp32
+    static constexpr size_t SMEM = REGION + DONE + 1024;
 };
+
+// One column step of the panel factorization: v[0] is the active column and
+// sc[p-1] the broadcast entry of panel column k + p.  v[p-1] <- v[p] - a sc[p-1]
+// (update and shift in one FMA) for the R columns that can still be live.
+template <int R>
+__device__ __forceinline__ void update_shift(float (&v)[64], float a, const float *sc) {
+#pragma unroll
+    for (int q = 0; q < (R + 1) / 4; ++q) {
+        const float4 s4 = reinterpret_cast<const float4 *>(sc)[q];
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int p = 4 * q + i + 1;
+            if (p <= R) v[p - 1] = fmaf(-a, sv[i], v[p]);
+        }
+    }
+}
+
+// Same, updating only p <= plim (the other live columns are just shifted).
+template <int R>
+__device__ __forceinline__ void update_shift_lim(float (&v)[64], float a, const float *sc, int plim) {
+#pragma unroll
+    for (int q = 0; q < (R + 1) / 4; ++q) {
+        const float4 s4 = reinterpret_cast<const float4 *>(sc)[q];
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int p = 4 * q + i + 1;
+            if (p <= R) v[p - 1] = p <= plim ? fmaf(-a, sv[i], v[p]) : v[p];
+        }
+    }
+}
 
 // Six piece products of a three-way split (dropped terms are below 2^-24):
 // hi.hi, hi.mid, mid.hi, hi.lo, lo.hi, mid.mid.
@@ -116,12 +149,14 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[2];
     __shared__ uint32_t tmem_base;
-    __shared__ float s_col[64];
-    __shared__ float s_e;
+    __shared__ __align__(16) float s_col[2][128];   // broadcast column entries, pre-shifted (double buffered)
+    __shared__ float s_e[2];            // next diagonal excess (double buffered)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int blk = warp >> 2, lb = (warp & 3) * 32;
     const int row = blk * 128 + lb + lane;
     const uint32_t region = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    float *done = reinterpret_cast<float *>(smraw + (region - tc::smem_u32(smraw)) + TmemChol::REGION);
+    for (int e = tid; e < 2 * 128; e += TmemChol::NT) (&s_col[0][0])[e] = 0.f;
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
         tc::mbar_init(&mbar[0], 1);
@@ -244,42 +279,50 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 for (int k = 0; k < 64; ++k)
                     if (j0 + k > row) v[k] = 0.f;
             }
-#pragma unroll
-            for (int k = 0; k < 64; ++k) {
-                if (k < nb) {
-                    const int kk = j0 + k;
-                    if (row == kk) s_e = v[k];
-                    __syncthreads();
-                    const float e = s_e;
-                    const float l = sqrtf(1.f + e);
-                    float a;
-                    if (row == kk) {
-                        v[k] = l;
-                        a = 1.f / l;
-                        if (!FACTOR) dR[start + kk] = 0.5f * log1pf(e);
-                    } else {
-                        v[k] = v[k] / l;
-                        a = v[k];
-                    }
-                    if (row > kk && row < j0 + 64) s_col[row - j0] = v[k];
-                    __syncthreads();
-                    if (!FACTOR) {
-                        if (row > kk) {
-#pragma unroll
-                            for (int p = k + 1; p < 64; ++p) v[p] = fmaf(-a, s_col[p], v[p]);
-                        }
-                    } else if (row > kk) {
-                        // L role: only this row's lower part (its upper part holds B, and B_i,kk = 0)
-#pragma unroll
-                        for (int p = k + 1; p < 64; ++p)
-                            if (j0 + p <= row) v[p] = fmaf(-a, s_col[p], v[p]);
-                    } else {
-                        // B role (row <= kk): B_i,p -= B_i,kk L_p,kk, with B_ii = 1 / L_ii
-#pragma unroll
-                        for (int p = k + 1; p < 64; ++p) v[p] = fmaf(-a, s_col[p], v[p]);
-                    }
+            // ---- factor the panel: compact column loop, one barrier per column.  The owner of
+            // the next diagonal folds this column into it before the barrier and publishes it.
+            const int rel = row - j0;
+            if (rel == 0) s_e[0] = v[0];
+            __syncthreads();
+#pragma unroll 1
+            for (int k = 0; k < nb; ++k) {
+                const int kk = j0 + k;
+                const float e = s_e[k & 1];
+                const float rl = rsqrtf(1.f + e);            // 1 / L_kk
+                float a, dv;
+                if (row == kk) {
+                    a = rl;                                  // B_kk: used by this row's B role
+                    dv = (1.f + e) * rl;                     // L_kk
+                    if (!FACTOR) dR[start + kk] = 0.5f * log1pf(e);
+                } else {
+                    a = v[0] * rl;                           // L_row,kk or (FACTOR, row < kk) B_row,kk
+                    dv = a;
+                }
+                done[row * 65 + k] = dv;
+                if (rel > k && rel < 64) s_col[k & 1][rel - k - 1] = a;
+                if (rel == k + 1 && k + 1 < nb) s_e[(k + 1) & 1] = fmaf(-a, a, v[1]);
+                __syncthreads();
+                const float *sc = &s_col[k & 1][0];          // sc[p-1] <-> panel column k + p
+                // INSEG: rows at or above the diagonal are finished.  FACTOR: rows of the diagonal
+                // block in the L role touch only their lower part (their upper part holds B and
+                // B_row,kk = 0); every other row updates all live columns.
+                if (!FACTOR && rel <= k) continue;
+                const bool lim = FACTOR && rel > k && rel < 64;
+                if (lim) {
+                    const int plim = rel - k;
+                    if (k < 16) update_shift_lim<63>(v, a, sc, plim);
+                    else if (k < 32) update_shift_lim<47>(v, a, sc, plim);
+                    else if (k < 48) update_shift_lim<31>(v, a, sc, plim);
+                    else update_shift_lim<15>(v, a, sc, plim);
+                } else {
+                    if (k < 16) update_shift<63>(v, a, sc);
+                    else if (k < 32) update_shift<47>(v, a, sc);
+                    else if (k < 48) update_shift<31>(v, a, sc);
+                    else update_shift<15>(v, a, sc);
                 }
             }
+#pragma unroll
+            for (int k = 0; k < 64; ++k) v[k] = k < nb ? done[row * 65 + k] : 0.f;
             // operand rows: FACTOR rows < j1 carry B (0 below the diagonal, 1/L_ii on it),
             // INSEG rows < j1 are not updated (zero); rows >= j1 carry L.
             if (row < j1) {
