@@ -7,9 +7,10 @@
 //
 // Positions are classified (chunk, bin), counted per bin and permuted so that
 // each bin's positions are contiguous; the product is then a grouped GEMM over
-// bins whose A rows are gathered chunk vectors and whose output rows are
-// scattered back to their positions with the residual added.
+// bins on tcgen05 whose A rows are gathered chunk vectors and whose output rows
+// are scattered back to their positions with the residual added.
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace dbc {
 namespace up {
@@ -100,81 +101,202 @@ __global__ void scan_bins_kernel(int nbins, Layout L) {
             L.tile_start[b] = t;
             L.cursor[b] = 0;
             s += L.hist[b];
-            t += (L.hist[b] + 63) / 64;
+            t += (L.hist[b] + 127) / 128;
         }
         L.bin_start[nbins] = s;
         L.tile_start[nbins] = t;
     }
 }
 
-__global__ void __launch_bounds__(256) scatter_kernel(int64_t N, Layout L) {
-    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < N;
-         p += (int64_t)gridDim.x * blockDim.x) {
-        const int b = L.bin[p];
-        const int slot = atomicAdd(&L.cursor[b], 1);
-        L.perm[L.bin_start[b] + slot] = (int32_t)p;
+// Positions -> their bin's slice of the permutation.  Slots are reserved per
+// block (one global atomic per bin and block), then handed out in shared memory.
+__global__ void __launch_bounds__(256) scatter_kernel(int64_t N, int nbins, Layout L) {
+    __shared__ int32_t cnt[kMaxBins], base[kMaxBins];
+    for (int64_t p0 = (int64_t)blockIdx.x * blockDim.x; p0 < N; p0 += (int64_t)gridDim.x * blockDim.x) {
+        for (int b = threadIdx.x; b < nbins; b += blockDim.x) cnt[b] = 0;
+        __syncthreads();
+        const int64_t p = p0 + threadIdx.x;
+        int b = -1, slot = 0;
+        if (p < N) {
+            b = L.bin[p];
+            slot = atomicAdd(&cnt[b], 1);
+        }
+        __syncthreads();
+        for (int q = threadIdx.x; q < nbins; q += blockDim.x)
+            base[q] = cnt[q] ? atomicAdd(&L.cursor[q], cnt[q]) : 0;
+        __syncthreads();
+        if (b >= 0) L.perm[L.bin_start[b] + base[b] + slot] = (int32_t)p;
+        __syncthreads();
     }
 }
 
-// Grouped GEMM tile: 64 positions of one bin x 64 output columns.
+// Grouped GEMM on tcgen05: one CTA = 128 positions of one bin x up to 256
+// output columns.  A = the positions' chunk vectors g_c (gathered rows,
+// K-major), B = W_b (row-major [d_g][d_l], read MN-major), fp32 accumulators
+// in TMEM; the epilogue adds h_t and scatters the rows back to their positions.
+struct BinTC {
+    static constexpr int NS = 3;
+    static constexpr uint32_t A_BYTES = 128 * 128;
+    static constexpr uint32_t B_BYTES = 4 * 64 * 128;          // up to 256 columns x 64 K, MN-major
+    static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+};
+
 template <class IN>
-__global__ void __launch_bounds__(256) bin_gemm_kernel(const __nv_bfloat16 *__restrict__ G, int64_t dg,
-                                                       const IN *__restrict__ H, int64_t dl,
-                                                       const __nv_bfloat16 *__restrict__ W, int nbins,
-                                                       Layout L, float *__restrict__ S) {
+__global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16 *__restrict__ G, int64_t dg,
+                                                             const IN *__restrict__ H, int64_t dl,
+                                                             const __nv_bfloat16 *__restrict__ W, int nbins,
+                                                             Layout L, float *__restrict__ S, int32_t *st) {
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[BinTC::NS];
+    __shared__ uint32_t tmem_base;
+    __shared__ int32_t pos[128], grow[128];
     const int tile = blockIdx.x;
     if (tile >= L.tile_start[nbins]) return;
     int b = 0;
     while (b + 1 < nbins && L.tile_start[b + 1] <= tile) ++b;
-    const int r0 = L.bin_start[b] + (tile - L.tile_start[b]) * 64;
-    const int cnt = min(64, L.bin_start[b + 1] - r0);
-    const int64_t n0 = (int64_t)blockIdx.y * 64;
-    __shared__ int32_t pos[64];
-    __shared__ int32_t grow[64];
-    __shared__ float As[32][65];
-    __shared__ float Bs[32][64];
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-    if (tid < 64) {
+    const int r0 = L.bin_start[b] + (tile - L.tile_start[b]) * 128;
+    const int cnt = min(128, L.bin_start[b + 1] - r0);
+    const int64_t n0 = (int64_t)blockIdx.y * 256;
+    const int nt = (int)(dl - n0 < 256 ? dl - n0 : 256);      // multiple of 64
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    {
         const int p = tid < cnt ? L.perm[r0 + tid] : -1;
         pos[tid] = p;
         grow[tid] = p >= 0 ? L.chunk[p] : -1;
     }
+    const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
+    if (tid == 0) {
+        for (int i = 0; i < BinTC::NS; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
     __syncthreads();
-    const __nv_bfloat16 *Wb = W + (size_t)b * dg * dl;
-    float acc[4][4] = {};
-    for (int64_t k0 = 0; k0 < dg; k0 += 32) {
-        for (int e = tid; e < 64 * 32; e += 256) {
-            const int rr = e >> 5, kk = e & 31;
-            const int g = grow[rr];
-            As[kk][rr] = g >= 0 ? __bfloat162float(G[(int64_t)g * dg + k0 + kk]) : 0.f;
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    const __nv_bfloat16 *Wb = W + (size_t)b * dg * dl + n0;
+    const int nchunks = (int)(dg / 64);
+    const int nb8 = nt / 8;
+    auto load = [&](int c, uint32_t sa) {
+        const uint32_t sb = sa + BinTC::A_BYTES;
+        for (int e = tid; e < 128 * 8; e += 128) {
+            const int r = e >> 3, ch = e & 7;
+            const int g = grow[r];
+            const __nv_bfloat16 *src = G + (size_t)(g >= 0 ? g : 0) * dg + c * 64 + ch * 8;
+            tc::cp_async16(sa + tc::kmajor_off(r, ch * 8), src, g >= 0 ? 16u : 0u);
         }
-        for (int e = tid; e < 32 * 64; e += 256) {
-            const int kk = e >> 6, cc = e & 63;
-            Bs[kk][cc] = __bfloat162float(Wb[(k0 + kk) * dl + n0 + cc]);
+        for (int e = tid; e < 64 * nb8; e += 128) {
+            const int k = e / nb8, n8 = e - (e / nb8) * nb8;
+            tc::cp_async16(sb + tc::mnmajor_off(n8 * 8, k, 8192), Wb + (size_t)(c * 64 + k) * dl + n8 * 8, 16u);
         }
+    };
+    const uint32_t idesc = tc::idesc_bf16(128, nt, false, true);
+    bool ok = true;
+    for (int c = 0; c < BinTC::NS - 1; ++c) {
+        if (c < nchunks) load(c, base + (uint32_t)c * BinTC::STAGE);
+        tc::cp_async_commit();
+    }
+    for (int c = 0; c < nchunks; ++c) {
+        const int cn = c + BinTC::NS - 1;
+        if (cn < nchunks) {
+            if (cn >= BinTC::NS) ok &= tc::mbar_wait(&mbar[cn % BinTC::NS], (uint32_t)((cn / BinTC::NS) - 1) & 1u, st);
+            load(cn, base + (uint32_t)(cn % BinTC::NS) * BinTC::STAGE);
+        }
+        tc::cp_async_commit();
+        tc::cp_async_wait<BinTC::NS - 1>();
+        tc::fence_async_smem();
         __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-            float a[4], bb[4];
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t sa = base + (uint32_t)(c % BinTC::NS) * BinTC::STAGE, sb = sa + BinTC::A_BYTES;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) { a[q] = As[kk][ty * 4 + q]; bb[q] = Bs[kk][tx * 4 + q]; }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) acc[q][r] = fmaf(a[q], bb[r], acc[q][r]);
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tbase, tc::sdesc(sa + kk * 32, 16, 1024), tc::sdesc(sb + kk * 2048, 8192, 1024), idesc,
+                             (c > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_commit(&mbar[c % BinTC::NS]);
         }
         __syncthreads();
     }
+    if (nchunks > 0) ok &= tc::mbar_wait(&mbar[(nchunks - 1) % BinTC::NS], (uint32_t)((nchunks - 1) / BinTC::NS) & 1u, st);
+    ok = __syncthreads_and(ok) != 0;
+    tc::fence_after_sync();
+    if (ok) {
+        // TMEM -> shared tile [128][nt] (row stride 260 floats), then one coalesced row at a time
+        tc::cp_async_wait<0>();
+        __syncthreads();
+        float *tile = reinterpret_cast<float *>(smraw + (base - tc::smem_u32(smraw)));
+        constexpr int LDT = 260;
+        const int r = warp * 32 + lane;
+#pragma unroll 1
+        for (int c0 = 0; c0 < nt; c0 += 16) {
+            float v[16];
+            tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            float4 *d = reinterpret_cast<float4 *>(tile + r * LDT + c0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int p = pos[ty * 4 + q];
-        if (p < 0) continue;
+            for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        __syncthreads();
+        const int nvec = nt / 8;                                   // 8 columns per lane
+#pragma unroll 1
+        for (int rr = warp; rr < 128; rr += 4) {
+            const int p = pos[rr];
+            if (p < 0) continue;
+            for (int c8 = lane; c8 < nvec; c8 += 32) {
+                const float *t = tile + rr * LDT + c8 * 8;
+                const float4 a0 = *reinterpret_cast<const float4 *>(t);
+                const float4 a1 = *reinterpret_cast<const float4 *>(t + 4);
+                float h[8];
+                const IN *hrow = H + (size_t)p * dl + n0 + c8 * 8;
+                if (sizeof(IN) == 2) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(hrow);
+                    const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int64_t j = n0 + tx * 4 + r;
-            S[(int64_t)p * dl + j] = ld_f(H + (int64_t)p * dl + j) + acc[q][r];
+                    for (int i = 0; i < 8; ++i) h[i] = __bfloat162float(hb[i]);
+                } else {
+                    const float4 f0 = *reinterpret_cast<const float4 *>(hrow);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(hrow + 4);
+                    h[0] = f0.x; h[1] = f0.y; h[2] = f0.z; h[3] = f0.w;
+                    h[4] = f1.x; h[5] = f1.y; h[6] = f1.z; h[7] = f1.w;
+                }
+                float4 *dst = reinterpret_cast<float4 *>(S + (size_t)p * dl + n0 + c8 * 8);
+                dst[0] = make_float4(a0.x + h[0], a0.y + h[1], a0.z + h[2], a0.w + h[3]);
+                dst[1] = make_float4(a1.x + h[4], a1.y + h[5], a1.z + h[6], a1.w + h[7]);
+            }
         }
     }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 256);
+}
+
+// Launch sequence shared by the workspace and the allocation-free entry points.
+inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, const int64_t *offsets, int64_t T,
+                         int64_t N, int64_t d_l, const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
+                         const void *W_bin, int nbins, int mode, float *S, const Layout &L, int32_t *dev_status,
+                         cudaStream_t s) {
+    cudaMemsetAsync(L.hist, 0, sizeof(int32_t) * kMaxBins, s);
+    const int sms = num_sms();
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (int64_t)sms * 8));
+    classify_kernel<<<grid, 256, 0, s>>>(offsets, T, N, idx, idx_offsets, rows, nbins, mode, L, dev_status);
+    scan_bins_kernel<<<1, 32, 0, s>>>(nbins, L);
+    scatter_kernel<<<grid, 256, 0, s>>>(N, nbins, L);
+    dim3 g((unsigned)((N + 127) / 128 + nbins), (unsigned)((d_l + 255) / 256));
+    if (dtype == DBC_BF16) {
+        cudaFuncSetAttribute(bin_gemm_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)BinTC::SMEM);
+        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 128, BinTC::SMEM, s>>>(
+            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
+            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
+    } else {
+        cudaFuncSetAttribute(bin_gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)BinTC::SMEM);
+        bin_gemm_tc_kernel<float><<<g, 128, BinTC::SMEM, s>>>(
+            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
+            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
+    }
+    count_launches(4);
+    return launch_status();
 }
 
 }  // namespace up
@@ -206,25 +328,8 @@ extern "C" dbc_status chunk_upsample(const void *G, int64_t d_g, const void *H, 
     if (!ws || ws_bytes < need.bytes || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)))
         return DBC_ERR_WORKSPACE;
     const up::Layout L = up::carve(ws, N);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaMemsetAsync(L.hist, 0, sizeof(int32_t) * up::kMaxBins, s);
-    const int sms = num_sms();
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (int64_t)sms * 8));
-    up::classify_kernel<<<grid, 256, 0, s>>>(offsets, T, N, idx, idx_offsets, rows, nbins, mode, L,
-                                             dev_status);
-    up::scan_bins_kernel<<<1, 32, 0, s>>>(nbins, L);
-    up::scatter_kernel<<<grid, 256, 0, s>>>(N, L);
-    dim3 g((unsigned)((N + 63) / 64 + nbins), (unsigned)(d_l / 64));
-    if (dtype == DBC_BF16)
-        up::bin_gemm_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S);
-    else
-        up::bin_gemm_kernel<float><<<g, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S);
-    count_launches(4);
-    return launch_status();
+    return up::launch(G, d_g, H, dtype, offsets, T, N, d_l, idx, idx_offsets, rows, W_bin, nbins, mode, S, L,
+                      dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -288,24 +393,7 @@ extern "C" dbc_status chunk_upsample_noalloc(const void *G, int64_t d_g, const v
     const dbc_status ss = up::noalloc_scratch(&scratch);
     if (ss != DBC_OK) return ss;
     const up::Layout L = up::carve(scratch, N);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // The bin counters must start at zero; everything else is written before it is read.
-    cudaMemsetAsync(L.hist, 0, sizeof(int32_t) * up::kMaxBins, s);
-    const int sms = num_sms();
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (int64_t)sms * 8));
-    up::classify_kernel<<<grid, 256, 0, s>>>(offsets, T, N, idx, idx_offsets, rows, nbins, mode, L,
-                                             dev_status);
-    up::scan_bins_kernel<<<1, 32, 0, s>>>(nbins, L);
-    up::scatter_kernel<<<grid, 256, 0, s>>>(N, L);
-    dim3 g((unsigned)((N + 63) / 64 + nbins), (unsigned)(d_l / 64));
-    if (dtype == DBC_BF16)
-        up::bin_gemm_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S);
-    else
-        up::bin_gemm_kernel<float><<<g, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S);
-    count_launches(4);
-    return launch_status();
+    // launch() clears the bin counters, the only scratch that must start at zero.
+    return up::launch(G, d_g, H, dtype, offsets, T, N, d_l, idx, idx_offsets, rows, W_bin, nbins, mode, S, L,
+                      dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
