@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--impl", default="dbc", choices=["dbc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--rows", action="store_true",
+                    help="time every hot-path row on its own workload family (one JSON line per row)")
+    ap.add_argument("--reps", type=int, default=10)
     return ap.parse_args()
 
 
@@ -165,11 +168,117 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- per-row measurements
+def _time(fn, reps, flush, stream):
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(np.median(ts))
+
+
+def run_rows(args):
+    """Each row of the hot path timed on the workload family it is specified on."""
+    import torch
+    import workloads
+    import dynamic_byte_chunking_b200 as dbc
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    pk, src = peaks()
+    hbm, tf = pk.get("hbm_gbs", 6650.0), pk.get("bf16_tflops", 1590.0)
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def emit(row, fam, ms, **kv):
+        line = {"row": row, "workload": fam, "ms": ms, **kv, "peak_source": src}
+        print(json.dumps(line), flush=True)
+
+    for fam in ["tiny", "byteflow", "bytegen", "wide", "ragged"]:
+        w = workloads.make(fam)
+        H = bf(w.H_bits) if w.dtype == "bf16" else torch.from_numpy(w.H_bits).to(dev)
+        offs = torch.from_numpy(w.offsets).to(dev)
+        o = offs if not w.dense else None
+        N, d, rows, T = w.N, w.d, w.rows, w.T
+        ws = torch.empty(dbc.chunk_coding_rate_workspace(rows, T, N, d), dtype=torch.uint8, device=dev)
+        dR = torch.empty(N, dtype=torch.float32, device=dev)
+        Hx = H if o is not None else H.view(rows, T, d)
+        ms = _time(lambda: dbc.chunk_coding_rate(Hx, w.eps2, offsets=o, T=T, dR=dR, workspace=ws), args.reps,
+                   flush, stream)
+        fl = 4.0 * d * d * N
+        emit("A1 coding rate", fam, ms, positions_per_s=N / (ms * 1e-3), tflops=fl / (ms * 1e-3) / 1e12,
+             frac_bf16_peak=fl / (ms * 1e-3) / 1e12 / tf)
+        Kt = torch.from_numpy(w.K).to(dev)
+        total = int(np.minimum(w.K, w.lengths).sum())
+        idx = torch.empty(total, dtype=torch.int64, device=dev)
+        io = torch.empty(rows + 1, dtype=torch.int64, device=dev)
+        ms = _time(lambda: dbc.chunk_topk_select(dR, Kt, rows=rows, T=T, offsets=o, idx=idx, idx_offsets=io,
+                                                 total=total), args.reps, flush, stream)
+        by = N * 4 + total * 8
+        emit("A2 top-k", fam, ms, gbs=by / (ms * 1e-3) / 1e9, frac_hbm=by / (ms * 1e-3) / 1e9 / hbm)
+        Z = torch.empty(total, d, dtype=H.dtype, device=dev)
+        ms = _time(lambda: dbc.chunk_gather(H, idx, io, rows=rows, T=T, offsets=o, total=total, Z=Z), args.reps,
+                   flush, stream)
+        by = 2 * total * d * H.element_size()
+        emit("A3 gather", fam, ms, gbs=by / (ms * 1e-3) / 1e9, frac_hbm=by / (ms * 1e-3) / 1e9 / hbm)
+        G = Z
+        if w.W_proj is not None:
+            Wp = bf(w.W_proj)
+            dg = Wp.shape[1]
+            Zf = torch.empty(total, dg, dtype=torch.float32, device=dev)
+            Zb = torch.empty(total, dg, dtype=torch.bfloat16, device=dev)
+            ms = _time(lambda: dbc.chunk_gather(H, idx, io, rows=rows, T=T, offsets=o, total=total, Z=Z, W_proj=Wp,
+                                                Zp_f32=Zf, Zp_bf16=Zb), args.reps, flush, stream)
+            fl = 2.0 * total * d * dg
+            emit("A3 gather + W_proj", fam, ms, tflops=fl / (ms * 1e-3) / 1e12, frac_bf16_peak=fl / (ms * 1e-3) / 1e12 / tf)
+            G = Zb
+        if w.W_bin is not None:
+            Wb = bf(w.W_bin)
+            nb, dg, dl = Wb.shape
+            S = torch.empty(N, dl, dtype=torch.float32, device=dev)
+            wsu = torch.empty(dbc.chunk_upsample_workspace(rows, N, nb), dtype=torch.uint8, device=dev)
+            ms = _time(lambda: dbc.chunk_upsample(G, H, idx, io, Wb, rows=rows, T=T, offsets=o, S=S, workspace=wsu),
+                       args.reps, flush, stream)
+            by = N * dl * H.element_size() + total * dg * 2 + nb * dg * dl * 2 + N * dl * 4
+            fl = 2.0 * N * dg * dl
+            emit("A4 upsample", fam, ms, gbs=by / (ms * 1e-3) / 1e9, frac_hbm=by / (ms * 1e-3) / 1e9 / hbm,
+                 tflops=fl / (ms * 1e-3) / 1e12)
+        if w.Wq is not None:
+            Wq, Wk = bf(w.Wq), bf(w.Wk)
+            wsr = torch.empty(dbc.hnet_route_workspace(rows, N, d), dtype=torch.uint8, device=dev)
+            ms = _time(lambda: dbc.hnet_route(H, Wq, Wk, offsets=offs, T=T, do_ema=False, workspace=wsr), args.reps,
+                       flush, stream)
+            fl = 4.0 * N * d * d
+            emit("A5 router", fam, ms, tflops=fl / (ms * 1e-3) / 1e12, frac_bf16_peak=fl / (ms * 1e-3) / 1e12 / tf)
+            ms2 = _time(lambda: dbc.hnet_route(H, Wq, Wk, offsets=offs, T=T, do_ema=True, workspace=wsr), args.reps,
+                        flush, stream)
+            p, b, ci, co, z = dbc.hnet_route(H, Wq, Wk, offsets=offs, T=T, do_ema=True, workspace=wsr)
+            nchunks = int(co[-1].item())
+            by = nchunks * d * (H.element_size() + 4) + nchunks * 12
+            emit("A6 EMA (router + EMA minus router)", fam, ms2 - ms, chunks=nchunks,
+                 gbs=by / max((ms2 - ms) * 1e-3, 1e-9) / 1e9)
+        del w, H, offs, ws, dR
+        torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------- device arm
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.rows:
+        run_rows(args)
         return
     import torch
     import workloads

@@ -5,6 +5,7 @@
 // vector loads/stores.  The projection is a bf16 GEMM with fp32 accumulation.
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 
 namespace dbc {
 namespace ga {
@@ -61,10 +62,17 @@ extern "C" dbc_status chunk_gather(const void *H, int dtype, const int64_t *offs
                                            dev_status);
     count_launches(W_proj ? 2 : 1);
     if (W_proj) {
-        dim3 g((unsigned)((total_K + 63) / 64), (unsigned)((d_g + 63) / 64));
-        gemm_bf16_simt<RowIdentity><<<g, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(Z), d, static_cast<const __nv_bfloat16 *>(W_proj), d_g,
-            Zp_f32, d_g, static_cast<__nv_bfloat16 *>(Zp_bf16), d_g, total_K, d_g, d, RowIdentity{});
+        const __nv_bfloat16 *Zb = static_cast<const __nv_bfloat16 *>(Z);
+        const __nv_bfloat16 *Wp = static_cast<const __nv_bfloat16 *>(W_proj);
+        if (d % 64 == 0 && d_g % 64 == 0) {
+            gt::launch_gemm_tc(Zb, d, Wp, d_g, Zp_f32, d_g, static_cast<__nv_bfloat16 *>(Zp_bf16), d_g, total_K, d_g,
+                               d, dev_status, s);
+        } else {
+            dim3 g((unsigned)((total_K + 63) / 64), (unsigned)((d_g + 63) / 64));
+            gemm_bf16_simt<RowIdentity><<<g, 256, 0, s>>>(Zb, d, Wp, d_g, Zp_f32, d_g,
+                                                          static_cast<__nv_bfloat16 *>(Zp_bf16), d_g, total_K, d_g,
+                                                          d, RowIdentity{});
+        }
     }
     return launch_status();
 }

@@ -10,21 +10,31 @@
 //   zbar_j = P_j h_{t_j} + (1 - P_j) zbar_{j-1} with P_j = p_{t_j}.
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "tc.cuh"
 
 namespace dbc {
 namespace rt {
 
+constexpr int kEmaBlk = 64;   // chunks per scan block
+
 struct Layout {
-    float *qk;        // [N, 2d]: q in columns [0, d), k in [d, 2d)
+    float *qk;        // [N, 2d]: q in columns [0, d), k in [d, 2d)   (d > 256 only)
     int64_t *count;   // [rows]
+    float *ema_a;     // [nblk, d] per-block affine map z_out = a z_in + b
+    float *ema_b;     // [nblk, d]
+    float *ema_z;     // [nblk, d] value entering each block
     size_t bytes;
 };
 
 inline Layout carve(void *ws, int64_t rows, int64_t N, int64_t d) {
     Carver c(ws);
     Layout L;
-    L.qk = c.take<float>((size_t)N * 2 * d);
+    L.qk = c.take<float>(d > 256 ? (size_t)N * 2 * d : 0);   // fp32 q|k only for the d > 256 path
     L.count = c.take<int64_t>(rows + 1);
+    const int64_t nblk = N / kEmaBlk + 1;
+    L.ema_a = c.take<float>((size_t)nblk * d);
+    L.ema_b = c.take<float>((size_t)nblk * d);
+    L.ema_z = c.take<float>((size_t)nblk * d);
     L.bytes = c.off;
     return L;
 }
@@ -64,6 +74,143 @@ __global__ void __launch_bounds__(256) prob_kernel(const float *__restrict__ qk,
             bnd[i] = pv >= threshold ? 1 : 0;
         }
     }
+}
+
+// q/k projections on tcgen05 with the cosine epilogue fused.  One CTA = 128
+// consecutive positions r0 .. r0+127.  The K-projection reads the rows shifted
+// by one (r0-1 .. r0+126), so TMEM lane i holds q_{r0+i} in columns [0, D) and
+// k_{r0+i-1} in columns [D, 2D): every thread finishes its own position.
+template <int D>
+struct RouterTC {
+    static constexpr int NS = 2;
+    static constexpr uint32_t A_BYTES = 128 * 128;
+    static constexpr uint32_t W_BYTES = D * 128;              // 64 K-rows x D columns, MN-major
+    static constexpr uint32_t STAGE = 2 * A_BYTES + 2 * W_BYTES;
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+    static constexpr int TCOLS = 2 * D < 32 ? 32 : 2 * D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1) router_tc_kernel(const __nv_bfloat16 *__restrict__ H,
+                                                           const int64_t *offsets, int64_t rows, int64_t T,
+                                                           int64_t N, const __nv_bfloat16 *__restrict__ Wq,
+                                                           const __nv_bfloat16 *__restrict__ Wk, float threshold,
+                                                           float *p, uint8_t *bnd, int32_t *st) {
+    using C = RouterTC<D>;
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[C::NS];
+    __shared__ uint32_t tmem_base;
+    const int64_t r0 = (int64_t)blockIdx.x * 128;
+    if (r0 >= N) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, C::TCOLS);
+    if (tid == 0) {
+        for (int i = 0; i < C::NS; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    constexpr int NCH = D / 64, NB8 = D / 8;
+    auto load = [&](int c, uint32_t sa) {
+        for (int e = tid; e < 2 * 128 * 8; e += 128) {
+            const int which = e >> 10, r = (e >> 3) & 127, ch = e & 7;
+            const int64_t t = r0 + r - which;                  // which = 1: shifted rows for k
+            const bool in = t >= 0 && t < N;
+            tc::cp_async16(sa + which * C::A_BYTES + tc::kmajor_off(r, ch * 8),
+                           H + (in ? t : 0) * D + c * 64 + ch * 8, in ? 16u : 0u);
+        }
+        const uint32_t sw = sa + 2 * C::A_BYTES;
+        for (int e = tid; e < 2 * 64 * NB8; e += 128) {
+            const int which = e / (64 * NB8), rem = e - which * (64 * NB8);
+            const int k = rem / NB8, n8 = rem - (rem / NB8) * NB8;
+            const __nv_bfloat16 *W = which ? Wk : Wq;
+            tc::cp_async16(sw + which * C::W_BYTES + tc::mnmajor_off(n8 * 8, k, 8192),
+                           W + (size_t)(c * 64 + k) * D + n8 * 8, 16u);
+        }
+    };
+    constexpr uint32_t idesc = tc::idesc_bf16(128, D, false, true);
+    bool ok = true;
+    for (int c = 0; c < C::NS - 1; ++c) {
+        if (c < NCH) load(c, base + (uint32_t)c * C::STAGE);
+        tc::cp_async_commit();
+    }
+    for (int c = 0; c < NCH; ++c) {
+        const int cn = c + C::NS - 1;
+        if (cn < NCH) {
+            if (cn >= C::NS) ok &= tc::mbar_wait(&mbar[cn % C::NS], (uint32_t)((cn / C::NS) - 1) & 1u, st);
+            load(cn, base + (uint32_t)(cn % C::NS) * C::STAGE);
+        }
+        tc::cp_async_commit();
+        tc::cp_async_wait<C::NS - 1>();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t sa = base + (uint32_t)(c % C::NS) * C::STAGE, sw = sa + 2 * C::A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+                tc::mma_bf16(tbase, tc::sdesc(sa + kk * 32, 16, 1024), tc::sdesc(sw + kk * 2048, 8192, 1024), idesc,
+                             acc);
+                tc::mma_bf16(tbase + D, tc::sdesc(sa + C::A_BYTES + kk * 32, 16, 1024),
+                             tc::sdesc(sw + C::W_BYTES + kk * 2048, 8192, 1024), idesc, acc);
+            }
+            tc::mma_commit(&mbar[c % C::NS]);
+        }
+        __syncthreads();
+    }
+    ok &= tc::mbar_wait(&mbar[(NCH - 1) % C::NS], (uint32_t)((NCH - 1) / C::NS) & 1u, st);
+    ok = __syncthreads_and(ok) != 0;
+    tc::fence_after_sync();
+    if (ok) {
+        const int64_t t = r0 + warp * 32 + lane;
+        float dot = 0.f, nq = 0.f, nk = 0.f;
+        const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float q[16], k[16];
+            tc::tmem_ld16(tl + (uint32_t)c0, q);
+            tc::tmem_ld16(tl + (uint32_t)(D + c0), k);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                dot = fmaf(q[i], k[i], dot);
+                nq = fmaf(q[i], q[i], nq);
+                nk = fmaf(k[i], k[i], nk);
+            }
+        }
+        if (t < N) {
+            bool first;
+            if (offsets) {
+                const int64_t r = find_row(offsets, rows, t);
+                first = offsets[r] == t;
+            } else {
+                first = (t % T) == 0;
+            }
+            float pv = 1.f;
+            if (!first) {
+                const float cs = (nq > 0.f && nk > 0.f) ? dot / (sqrtf(nq) * sqrtf(nk)) : 0.f;
+                pv = 0.5f * (1.f - cs);
+            }
+            if (!isfinite(pv)) flag(st, DBC_ERR_NONFINITE);
+            p[t] = pv;
+            bnd[t] = pv >= threshold ? 1 : 0;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, C::TCOLS);
+}
+
+template <int D>
+void launch_router_tc(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N,
+                      const __nv_bfloat16 *Wq, const __nv_bfloat16 *Wk, float threshold, float *p, uint8_t *b,
+                      int32_t *st, cudaStream_t s) {
+    cudaFuncSetAttribute(router_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RouterTC<D>::SMEM);
+    router_tc_kernel<D><<<(unsigned)((N + 127) / 128), 128, RouterTC<D>::SMEM, s>>>(H, offsets, rows, T, N, Wq, Wk,
+                                                                                   threshold, p, b, st);
 }
 
 __device__ __forceinline__ int64_t block_scan_excl(int64_t v, int64_t *wsum, int64_t *total) {
@@ -143,24 +290,77 @@ __global__ void __launch_bounds__(1024) compact_kernel(const uint8_t *bnd, const
     }
 }
 
-// One thread per (row, feature): sequential over the row's chunks.
-template <class IN>
-__global__ void __launch_bounds__(256) ema_kernel(const IN *__restrict__ H, const int64_t *offsets,
-                                                  int64_t rows, int64_t T, int64_t d, const float *p,
-                                                  const int64_t *co, const int64_t *chunk_idx, float *z) {
-    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (g >= rows * d) return;
-    const int64_t r = g / d, f = g - (g / d) * d;
+// EMA over the rows-stacked chunk list as one sequence: p = 1 at every row's
+// first position, so the recurrence restarts there by itself.  Three passes:
+// per 64-chunk block the affine map z_out = a z_in + b (parallel over blocks
+// and features), the chain of block maps, then the recomputation inside blocks.
+__device__ __forceinline__ void chunk_source(const int64_t *offsets, int64_t rows, int64_t T, const int64_t *co,
+                                             const int64_t *chunk_idx, int64_t j, int64_t &pos) {
+    const int64_t r = find_row(co, rows, j);
     int64_t a, n;
     row_bounds(offsets, r, T, a, n);
-    const int64_t c0 = co[r], c1 = co[r + 1];
-    float acc = 0.f;
-    for (int64_t j = c0; j < c1; ++j) {
-        const int64_t t = a + chunk_idx[j];
-        const float P = p[t];
-        const float x = ld_f(H + t * d + f);
-        acc = P * x + (1.f - P) * acc;
-        z[j * d + f] = acc;
+    pos = a + chunk_idx[j];
+}
+
+template <class IN, bool FINAL>
+__global__ void __launch_bounds__(256) ema_block_kernel(const IN *__restrict__ H, const int64_t *offsets,
+                                                        int64_t rows, int64_t T, int64_t d, const float *p,
+                                                        const int64_t *co, const int64_t *chunk_idx, Layout L,
+                                                        float *z) {
+    __shared__ int64_t spos[kEmaBlk];
+    __shared__ float sP[kEmaBlk];
+    const int64_t total = co[rows];
+    const int64_t j0 = (int64_t)blockIdx.x * kEmaBlk;
+    if (j0 >= total) return;
+    const int cnt = (int)(total - j0 < kEmaBlk ? total - j0 : kEmaBlk);
+    if (threadIdx.x < cnt) {
+        int64_t pos;
+        chunk_source(offsets, rows, T, co, chunk_idx, j0 + threadIdx.x, pos);
+        spos[threadIdx.x] = pos;
+        sP[threadIdx.x] = p[pos];
+    }
+    __syncthreads();
+    for (int64_t f = threadIdx.x; f < d; f += blockDim.x) {
+        if (!FINAL) {
+            float a = 1.f, b = 0.f;
+            for (int j = 0; j < cnt; ++j) {
+                const float P = sP[j];
+                a = (1.f - P) * a;
+                b = P * ld_f(H + spos[j] * d + f) + (1.f - P) * b;
+            }
+            L.ema_a[blockIdx.x * d + f] = a;
+            L.ema_b[blockIdx.x * d + f] = b;
+        } else {
+            float acc = L.ema_z[blockIdx.x * d + f];
+            for (int j = 0; j < cnt; ++j) {
+                const float P = sP[j];
+                acc = P * ld_f(H + spos[j] * d + f) + (1.f - P) * acc;
+                z[(j0 + j) * d + f] = acc;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) ema_chain_kernel(int64_t rows, int64_t d, const int64_t *co, Layout L) {
+    const int64_t total = co[rows];
+    const int64_t nblk = (total + kEmaBlk - 1) / kEmaBlk;
+    const int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (f >= d) return;
+    float zc = 0.f;
+    int64_t b = 0;
+    for (; b + 4 <= nblk; b += 4) {
+        float a[4], bb[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { a[q] = L.ema_a[(b + q) * d + f]; bb[q] = L.ema_b[(b + q) * d + f]; }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            L.ema_z[(b + q) * d + f] = zc;
+            zc = a[q] * zc + bb[q];
+        }
+    }
+    for (; b < nblk; ++b) {
+        L.ema_z[b * d + f] = zc;
+        zc = L.ema_a[b * d + f] * zc + L.ema_b[b * d + f];
     }
 }
 
@@ -195,23 +395,34 @@ extern "C" dbc_status hnet_route(const void *H, const int64_t *offsets, int64_t 
         return DBC_ERR_WORKSPACE;
     const rt::Layout L = rt::carve(ws, rows, N, d);
     const __nv_bfloat16 *Hb = static_cast<const __nv_bfloat16 *>(H);
-    dim3 g((unsigned)((N + 63) / 64), (unsigned)(d / 64));
-    gemm_bf16_simt<RowIdentity><<<g, 256, 0, s>>>(Hb, d, static_cast<const __nv_bfloat16 *>(Wq), d,
-                                                  L.qk, 2 * d, nullptr, 0, N, d, d, RowIdentity{});
-    gemm_bf16_simt<RowIdentity><<<g, 256, 0, s>>>(Hb, d, static_cast<const __nv_bfloat16 *>(Wk), d,
-                                                  L.qk + d, 2 * d, nullptr, 0, N, d, d, RowIdentity{});
-    const int sms = num_sms();
-    const int pg = (int)std::max<int64_t>(1, std::min<int64_t>((N + 7) / 8, (int64_t)sms * 32));
-    rt::prob_kernel<<<pg, 256, 0, s>>>(L.qk, offsets, rows, T, N, d, threshold, p, boundary, dev_status);
+    const __nv_bfloat16 *Wqb = static_cast<const __nv_bfloat16 *>(Wq), *Wkb = static_cast<const __nv_bfloat16 *>(Wk);
+    if (d <= 256) {
+        switch (d) {
+            case 64: rt::launch_router_tc<64>(Hb, offsets, rows, T, N, Wqb, Wkb, threshold, p, boundary, dev_status, s); break;
+            case 128: rt::launch_router_tc<128>(Hb, offsets, rows, T, N, Wqb, Wkb, threshold, p, boundary, dev_status, s); break;
+            default: rt::launch_router_tc<256>(Hb, offsets, rows, T, N, Wqb, Wkb, threshold, p, boundary, dev_status, s);
+        }
+    } else {
+        dim3 g((unsigned)((N + 63) / 64), (unsigned)(d / 64));
+        gemm_bf16_simt<RowIdentity><<<g, 256, 0, s>>>(Hb, d, Wqb, d, L.qk, 2 * d, nullptr, 0, N, d, d, RowIdentity{});
+        gemm_bf16_simt<RowIdentity><<<g, 256, 0, s>>>(Hb, d, Wkb, d, L.qk + d, 2 * d, nullptr, 0, N, d, d,
+                                                      RowIdentity{});
+        const int sms = num_sms();
+        const int pg = (int)std::max<int64_t>(1, std::min<int64_t>((N + 7) / 8, (int64_t)sms * 32));
+        rt::prob_kernel<<<pg, 256, 0, s>>>(L.qk, offsets, rows, T, N, d, threshold, p, boundary, dev_status);
+    }
     const int rg = (int)std::min<int64_t>(rows, 65535);
     rt::count_kernel<<<rg, 1024, 0, s>>>(boundary, offsets, rows, T, L.count);
     rt::offsets_kernel<<<1, 1024, 0, s>>>(L.count, rows, chunk_offsets);
     rt::compact_kernel<<<rg, 1024, 0, s>>>(boundary, offsets, rows, T, chunk_offsets, chunk_idx);
-    count_launches(do_ema ? 7 : 6);
+    count_launches((d <= 256 ? 4 : 6) + (do_ema ? 3 : 0));
     if (do_ema) {
-        const int64_t th = rows * d;
-        rt::ema_kernel<__nv_bfloat16><<<(unsigned)((th + 255) / 256), 256, 0, s>>>(
-            Hb, offsets, rows, T, d, p, chunk_offsets, chunk_idx, z_smooth);
+        const unsigned nblk = (unsigned)(N / rt::kEmaBlk + 1);
+        rt::ema_block_kernel<__nv_bfloat16, false><<<nblk, 256, 0, s>>>(Hb, offsets, rows, T, d, p, chunk_offsets,
+                                                                        chunk_idx, L, z_smooth);
+        rt::ema_chain_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(rows, d, chunk_offsets, L);
+        rt::ema_block_kernel<__nv_bfloat16, true><<<nblk, 256, 0, s>>>(Hb, offsets, rows, T, d, p, chunk_offsets,
+                                                                       chunk_idx, L, z_smooth);
     }
     return launch_status();
 }

@@ -50,7 +50,11 @@ def test_workspace_queries_scale(L):
     b = dbc.chunk_coding_rate_workspace(16, 8192, 16 * 8192, 256)
     assert 0 < a < b
     assert dbc.chunk_upsample_workspace(8, 65536, 16) > 65536
-    assert dbc.hnet_route_workspace(64, 4096 * 64, 256) >= 4096 * 64 * 512 * 4
+    # d = 256: the projections are fused on tensor cores; scratch = EMA block maps (3 x nblk x d fp32)
+    N = 4096 * 64
+    assert dbc.hnet_route_workspace(64, N, 256) >= 3 * (N // 64) * 256 * 4
+    # d = 512 keeps an fp32 q|k buffer
+    assert dbc.hnet_route_workspace(64, N, 512) >= N * 1024 * 4
 
 
 def test_argument_errors_return_before_launch(L):
