@@ -8,7 +8,9 @@
 // sqrt(1 + e).
 //
 // Per 64-column panel: every thread loads its row's 64 panel entries with
-// tcgen05.ld, the panel is factored in registers (two barriers per column),
+// tcgen05.ld, the panel is factored in registers in 16-column sub-panels
+// (diagonal block by shuffles, then a solve and a rank-16 update per row:
+// two barriers per sub-panel),
 // the panel rows are split into three bf16 pieces (hi + mid + lo carries the
 // fp32 value) and staged in shared memory, and the trailing columns are
 // updated in place by tcgen05 MMAs with negated A over the six piece
@@ -41,35 +43,28 @@ struct TmemChol {
     static constexpr size_t SMEM = REGION + DONE + 1024;
 };
 
-// One column step of the panel factorization: v[0] is the active column and
-// sc[p-1] the broadcast entry of panel column k + p.  v[p-1] <- v[p] - a sc[p-1]
-// (update and shift in one FMA) for the R columns that can still be live.
-template <int R>
-__device__ __forceinline__ void update_shift(float (&v)[64], float a, const float *sc) {
+// Rank-16 update and shift of the live panel columns of one row:
+// v[p] <- v[16 + p] - sum_c a[c] L(p)[c] for p in [0, P), with L(p) the solved
+// sub-panel row of panel column (kb + 16 + p) in shared memory (stride 20).
+// Columns p > plim are only shifted (a row of the diagonal block in the L role
+// must not touch its upper part, which carries B in the factor mode).
+template <int P>
+__device__ __forceinline__ void rank16_shift(float (&v)[64], const float (&a)[16], const float *sL, int plim) {
 #pragma unroll
-    for (int q = 0; q < (R + 1) / 4; ++q) {
-        const float4 s4 = reinterpret_cast<const float4 *>(sc)[q];
-        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+    for (int p = 0; p < P; ++p) {
+        float x = v[16 + p];
+        if (p <= plim) {
+            const float4 *lr = reinterpret_cast<const float4 *>(sL + p * 20);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int p = 4 * q + i + 1;
-            if (p <= R) v[p - 1] = fmaf(-a, sv[i], v[p]);
+            for (int q = 0; q < 4; ++q) {
+                const float4 l = lr[q];
+                x = fmaf(-a[4 * q], l.x, x);
+                x = fmaf(-a[4 * q + 1], l.y, x);
+                x = fmaf(-a[4 * q + 2], l.z, x);
+                x = fmaf(-a[4 * q + 3], l.w, x);
+            }
         }
-    }
-}
-
-// Same, updating only p <= plim (the other live columns are just shifted).
-template <int R>
-__device__ __forceinline__ void update_shift_lim(float (&v)[64], float a, const float *sc, int plim) {
-#pragma unroll
-    for (int q = 0; q < (R + 1) / 4; ++q) {
-        const float4 s4 = reinterpret_cast<const float4 *>(sc)[q];
-        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int p = 4 * q + i + 1;
-            if (p <= R) v[p - 1] = p <= plim ? fmaf(-a, sv[i], v[p]) : v[p];
-        }
+        v[p] = x;
     }
 }
 
@@ -149,14 +144,15 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[2];
     __shared__ uint32_t tmem_base;
-    __shared__ __align__(16) float s_col[2][128];   // broadcast column entries, pre-shifted (double buffered)
-    __shared__ float s_e[2];            // next diagonal excess (double buffered)
+    __shared__ __align__(16) float s_L[64][20];     // solved sub-panel rows of the panel's rows (rank-16 update)
+    __shared__ __align__(16) float s_Ld[16][20];    // factored 16 x 16 diagonal block
+    __shared__ float s_rl[16];                      // 1 / L_kk of the diagonal block
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int blk = warp >> 2, lb = (warp & 3) * 32;
     const int row = blk * 128 + lb + lane;
     const uint32_t region = (tc::smem_u32(smraw) + 1023u) & ~1023u;
     float *done = reinterpret_cast<float *>(smraw + (region - tc::smem_u32(smraw)) + TmemChol::REGION);
-    for (int e = tid; e < 2 * 128; e += TmemChol::NT) (&s_col[0][0])[e] = 0.f;
+    for (int e = tid; e < 64 * 20; e += TmemChol::NT) (&s_L[0][0])[e] = 0.f;
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
         tc::mbar_init(&mbar[0], 1);
@@ -279,46 +275,81 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 for (int k = 0; k < 64; ++k)
                     if (j0 + k > row) v[k] = 0.f;
             }
-            // ---- factor the panel: compact column loop, one barrier per column.  The owner of
-            // the next diagonal folds this column into it before the barrier and publishes it.
+            // ---- factor the panel in 16-column sub-panels: (1) the 16 x 16 diagonal block by its
+            // half-warp with shuffles, (2) every other live row solves its 16 values against it,
+            // (3) rank-16 update of the later panel columns with a shift by 16, so the current
+            // sub-panel is always v[0..15].  Two barriers per sub-panel.
             const int rel = row - j0;
-            if (rel == 0) s_e[0] = v[0];
-            __syncthreads();
+            const int nsub = (nb + 15) / 16;
 #pragma unroll 1
-            for (int k = 0; k < nb; ++k) {
-                const int kk = j0 + k;
-                const float e = s_e[k & 1];
-                const float rl = rsqrtf(1.f + e);            // 1 / L_kk
-                float a, dv;
-                if (row == kk) {
-                    a = rl;                                  // B_kk: used by this row's B role
-                    dv = (1.f + e) * rl;                     // L_kk
-                    if (!FACTOR) dR[start + kk] = 0.5f * log1pf(e);
-                } else {
-                    a = v[0] * rl;                           // L_row,kk or (FACTOR, row < kk) B_row,kk
-                    dv = a;
+            for (int q = 0; q < nsub; ++q) {
+                const int kb = 16 * q;
+                const int ii = rel - kb;
+                const bool diag = ii >= 0 && ii < 16;
+                float a[16];
+                if (diag) {
+                    const int lb0 = lane & 16;
+                    const unsigned mask = 0xFFFFu << lb0;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const float e = __shfl_sync(mask, v[c], lb0 + c);
+                        const float rlc = rsqrtf(1.f + e);
+                        if (ii == c) {
+                            v[c] = (1.f + e) * rlc;                       // L_cc
+                            s_rl[c] = rlc;
+                            if (!FACTOR && kb + c < nb) dR[start + j0 + kb + c] = 0.5f * log1pf(e);
+                        } else if (ii > c) {
+                            v[c] *= rlc;                                  // L_ii,c
+                        }
+#pragma unroll
+                        for (int c2 = 0; c2 < 16; ++c2) {
+                            if (c2 > c) {
+                                const float l2 = __shfl_sync(mask, v[c], lb0 + c2);
+                                if (ii >= c2) v[c2] = fmaf(-v[c], l2, v[c2]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const float x = c <= ii ? v[c] : 0.f;
+                        s_Ld[ii][c] = x;
+                        if (c <= ii) done[row * 65 + kb + c] = x;
+                    }
                 }
-                done[row * 65 + k] = dv;
-                if (rel > k && rel < 64) s_col[k & 1][rel - k - 1] = a;
-                if (rel == k + 1 && k + 1 < nb) s_e[(k + 1) & 1] = fmaf(-a, a, v[1]);
                 __syncthreads();
-                const float *sc = &s_col[k & 1][0];          // sc[p-1] <-> panel column k + p
-                // INSEG: rows at or above the diagonal are finished.  FACTOR: rows of the diagonal
-                // block in the L role touch only their lower part (their upper part holds B and
-                // B_row,kk = 0); every other row updates all live columns.
-                if (!FACTOR && rel <= k) continue;
-                const bool lim = FACTOR && rel > k && rel < 64;
-                if (lim) {
-                    const int plim = rel - k;
-                    if (k < 16) update_shift_lim<63>(v, a, sc, plim);
-                    else if (k < 32) update_shift_lim<47>(v, a, sc, plim);
-                    else if (k < 48) update_shift_lim<31>(v, a, sc, plim);
-                    else update_shift_lim<15>(v, a, sc, plim);
-                } else {
-                    if (k < 16) update_shift<63>(v, a, sc);
-                    else if (k < 32) update_shift<47>(v, a, sc);
-                    else if (k < 48) update_shift<31>(v, a, sc);
-                    else update_shift<15>(v, a, sc);
+                const bool live = FACTOR || ii >= 16;        // INSEG rows at or above the block are done
+                if (live) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (diag && c <= ii) {
+                            a[c] = c == ii ? s_rl[c] : 0.f;         // B role of a diagonal-block row: B_ii = 1/L_ii
+                        } else {
+                            const float4 *lr = reinterpret_cast<const float4 *>(&s_Ld[c][0]);
+                            float x = v[c];
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const float4 l = lr[q4];
+                                if (4 * q4 + 0 < c) x = fmaf(-a[4 * q4 + 0], l.x, x);
+                                if (4 * q4 + 1 < c) x = fmaf(-a[4 * q4 + 1], l.y, x);
+                                if (4 * q4 + 2 < c) x = fmaf(-a[4 * q4 + 2], l.z, x);
+                                if (4 * q4 + 3 < c) x = fmaf(-a[4 * q4 + 3], l.w, x);
+                            }
+                            a[c] = x * s_rl[c];
+                            done[row * 65 + kb + c] = a[c];
+                        }
+                    }
+                    if (ii >= 16 && rel < 64) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) s_L[rel][c] = a[c];
+                    }
+                }
+                __syncthreads();
+                if (live && q + 1 < nsub) {
+                    const float *sL = &s_L[kb + 16][0];
+                    const int plim = (FACTOR && ii >= 16 && rel < 64) ? ii - 16 : 64;
+                    if (q == 0) rank16_shift<48>(v, a, sL, plim);
+                    else if (q == 1) rank16_shift<32>(v, a, sL, plim);
+                    else rank16_shift<16>(v, a, sL, plim);
                 }
             }
 #pragma unroll
