@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--rows", action="store_true",
                     help="time every hot-path row on its own workload family (one JSON line per row)")
     ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--traffic-from", default=None, metavar="CSV",
+                    help="convert an ncu --csv launch list with dram__bytes_read.sum and dram__bytes_write.sum "
+                         "(taken on this workload) into profiles/dram_traffic_byteflow.json, then exit")
     return ap.parse_args()
 
 
@@ -171,6 +174,46 @@ def stored_traffic(kernel):
         return t["bytes_per_call"].get(kernel)
     except Exception:
         return None
+
+
+# kernel-name prefixes of each C-ABI call's kernels
+STAGE_PREFIX = {"chunk_coding_rate": "cr::", "chunk_topk_select": "tk::", "chunk_gather": "ga::",
+                "chunk_upsample": "up::"}
+
+
+def write_traffic(csv_path):
+    """Sum DRAM bytes per C-ABI call from an ncu CSV launch list and store them with the source hash.
+
+    Each call's bytes are the sum over its kernels' launches divided by the number of times the
+    call's first kernel launched (one per step)."""
+    import csv
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(f)]
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    h = rows[hi]
+    ki, mi, vi, ui, ii = (h.index("Kernel Name"), h.index("Metric Name"), h.index("Metric Value"),
+                          h.index("Metric Unit"), h.index("ID"))
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    per_launch = {}
+    for r in rows[hi + 1:]:
+        if len(r) <= vi or r[mi] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        name = r[ki]
+        b = float(r[vi].replace(",", "")) * scale.get(r[ui], 1)
+        per_launch.setdefault(r[ii], [name, 0.0])[1] += b
+    out = {}
+    for stage, pre in STAGE_PREFIX.items():
+        launches = [(n, b) for n, b in per_launch.values() if pre in n]
+        if not launches:
+            continue
+        first = launches[0][0].split("(")[0]
+        calls = sum(1 for n, _ in launches if n.split("(")[0] == first)
+        out[stage] = sum(b for _, b in launches) / calls
+    path = os.path.join(ROOT, "profiles", "dram_traffic_byteflow.json")
+    with open(path, "w") as f:
+        json.dump({"csrc_sha256": csrc_sha256(), "source": os.path.basename(csv_path),
+                   "bytes_per_call": out}, f, indent=1)
+    print(json.dumps(out))
 
 
 def run_reference(args):
@@ -304,6 +347,9 @@ def run_rows(args):
 # ---------------------------------------------------------------- device arm
 def main():
     args = parse()
+    if args.traffic_from:
+        write_traffic(args.traffic_from)
+        return
     if args.impl == "reference":
         run_reference(args)
         return

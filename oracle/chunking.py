@@ -15,6 +15,13 @@ Sources (ByteFlow, arXiv 2603.03583):
   chunk length, ABSOLUTE b = floor(t B / T) (the summary's b = floor(t/(T/B)),
   0-based).
 
+Backward (gradients of the upsampling for training with the chunker; the
+selection itself passes no gradient, notes "Key design 2"): with dS = dL/dS,
+  dL/dg_k  = sum over t in chunk k of W_{b(t)} dS_t,
+  dL/dW_b  = sum over t in bin b of g_{c(t)} (outer) dS_t,
+  dL/dh_t  = dS_t (the residual), and through the gather z_k = h_{s_k} the
+  chunk gradient returns to the boundary rows, dL/dh_{s_k} += dL/dz_k.
+
 All positions are 0-based.  Test infrastructure only.
 """
 from __future__ import annotations
@@ -22,7 +29,8 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["topk_select", "topk_select_rows", "gather", "chunk_of", "bin_of",
-           "upsample_row", "upsample", "BIN_OFFSET", "BIN_FRACTION", "BIN_ABSOLUTE"]
+           "upsample_row", "upsample", "upsample_backward_row", "upsample_backward", "gather_backward",
+           "BIN_OFFSET", "BIN_FRACTION", "BIN_ABSOLUTE"]
 
 BIN_OFFSET, BIN_FRACTION, BIN_ABSOLUTE = 0, 1, 2
 
@@ -118,3 +126,50 @@ def upsample(G, H, offsets, idx, idx_offsets, W_bin, mode=BIN_OFFSET, rows=None)
         ia, ib = idx_offsets[r], idx_offsets[r + 1]
         outs.append(upsample_row(G[ia:ib], H[a:b], idx[ia:ib], W_bin, mode))
     return outs
+
+
+def upsample_backward_row(G: np.ndarray, idx_row: np.ndarray, W_bin: np.ndarray,
+                          dS: np.ndarray, mode: int):
+    """Gradients of one row's s_t = h_t + g_{c(t)} W_{b(t)} given dS_t, float64.
+
+    Returns (dG [K, d_g], dW [B, d_g, d_l] of this row, dH [T, d_l]).  One
+    position at a time, straight from the chain rule.
+    """
+    T = dS.shape[0]
+    B = W_bin.shape[0]
+    c = chunk_of(idx_row, T)
+    b = bin_of(idx_row, T, B, mode)
+    G = np.asarray(G, dtype=np.float64)
+    W = np.asarray(W_bin, dtype=np.float64)
+    dS = np.asarray(dS, dtype=np.float64)
+    dG = np.zeros_like(G)
+    dW = np.zeros_like(W)
+    for t in range(T):
+        dG[c[t]] += W[b[t]] @ dS[t]
+        dW[b[t]] += np.outer(G[c[t]], dS[t])
+    return dG, dW, dS.copy()
+
+
+def upsample_backward(G, offsets, idx, idx_offsets, W_bin, dS, mode=BIN_OFFSET):
+    """Packed batch: (dG [sum K, d_g], dW summed over rows, dH = dS)."""
+    dG = np.zeros(np.shape(G), dtype=np.float64)
+    dW = np.zeros(np.shape(W_bin), dtype=np.float64)
+    for r in range(len(offsets) - 1):
+        a, b = offsets[r], offsets[r + 1]
+        ia, ib = idx_offsets[r], idx_offsets[r + 1]
+        if ib == ia:
+            continue
+        g, w, _ = upsample_backward_row(G[ia:ib], idx[ia:ib], W_bin, dS[a:b], mode)
+        dG[ia:ib] = g
+        dW += w
+    return dG, dW, np.asarray(dS, dtype=np.float64).copy()
+
+
+def gather_backward(dZ, offsets, idx, idx_offsets, N):
+    """Adjoint of the gather: dH [N, d] with dH[offsets_r + s_k] = dZ_k, zero elsewhere."""
+    dZ = np.asarray(dZ, dtype=np.float64)
+    dH = np.zeros((N, dZ.shape[1]), dtype=np.float64)
+    for r in range(len(offsets) - 1):
+        a, b = idx_offsets[r], idx_offsets[r + 1]
+        dH[offsets[r] + idx[a:b]] += dZ[a:b]
+    return dH
