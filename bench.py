@@ -326,6 +326,30 @@ def run_rows(args):
             fl = 2.0 * N * dg * dl
             emit("A4 upsample", fam, ms, gbs=by / (ms * 1e-3) / 1e9, frac_hbm=by / (ms * 1e-3) / 1e9 / hbm,
                  tflops=fl / (ms * 1e-3) / 1e12)
+            if dg % 128 == 0:
+                # backward of the upsampling + the gather's adjoint (dH = dS + scatter of dG)
+                gen = torch.Generator(device=dev).manual_seed(7)
+                dS = torch.randn(N, dl, dtype=torch.float32, device=dev, generator=gen)
+                dG = torch.empty(total, dg, dtype=torch.float32, device=dev)
+                dW = torch.empty(nb, dg, dl, dtype=torch.float32, device=dev)
+                dH = torch.empty(N, dl, dtype=torch.float32, device=dev)
+                wsb = torch.empty(dbc.chunk_upsample_backward_workspace(rows, N, nb, dl), dtype=torch.uint8,
+                                  device=dev)
+
+                def bwd():
+                    dbc.chunk_upsample_backward(dS, G, idx, io, Wb, rows=rows, T=T, offsets=o, dG=dG, dW=dW, dH=dH,
+                                                workspace=wsb)
+                    if dg == dl and G is Z:
+                        dbc.chunk_gather_backward(dG, idx, io, rows=rows, T=T, dH=dH, offsets=o)
+
+                ms = _time(bwd, args.reps, flush, stream)
+                # algorithmic bytes: read dS, G, W; write dG, dW, dH (the scatter into dH re-reads and writes
+                # only boundary rows, counted once each way)
+                by = (N * dl * 4 + total * dg * 2 + nb * dg * dl * 2 + total * dg * 4 + nb * dg * dl * 4
+                      + N * dl * 4 + (2 * total * dl * 4 if dg == dl and G is Z else 0))
+                emit("NEXT-1 upsample + gather backward", fam, ms, gbs=by / (ms * 1e-3) / 1e9,
+                     frac_hbm=by / (ms * 1e-3) / 1e9 / hbm)
+                del dS, dG, dW, dH, wsb
         if w.Wq is not None:
             Wq, Wk = bf(w.Wq), bf(w.Wk)
             wsr = torch.empty(dbc.hnet_route_workspace(rows, N, d), dtype=torch.uint8, device=dev)

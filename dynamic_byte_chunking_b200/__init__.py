@@ -25,6 +25,7 @@ __all__ = [
     "DbcError", "lib", "lib_path", "version", "status_string", "launch_count",
     "chunk_coding_rate", "chunk_coding_rate_workspace", "chunk_topk_select",
     "chunk_gather", "chunk_upsample", "chunk_upsample_workspace", "chunk_upsample_noalloc",
+    "chunk_upsample_backward", "chunk_upsample_backward_workspace", "chunk_gather_backward",
     "hnet_route", "hnet_route_workspace", "chunk",
     "DBC_F32", "DBC_BF16", "BIN_OFFSET", "BIN_FRACTION", "BIN_ABSOLUTE",
     "ERR_NONFINITE", "ERR_TIMEOUT", "ERR_BOUNDS",
@@ -55,6 +56,10 @@ _SIGS = {
                               _int, _vp, _vp, _sz, _vp, _vp]),
     "chunk_upsample_noalloc": (_int, [_vp, _i64, _vp, _int, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp,
                                       _int, _int, _vp, _vp, _vp]),
+    "chunk_upsample_backward_workspace": (_sz, [_i64, _i64, _int, _i64]),
+    "chunk_upsample_backward": (_int, [_vp, _vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _int,
+                                       _int, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "chunk_gather_backward": (_int, [_vp, _i64, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _int, _vp, _vp]),
     "hnet_route_workspace": (_sz, [_i64, _i64, _i64]),
     "hnet_route": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _f32, _int, _vp, _vp, _vp, _vp,
                           _vp, _vp, _sz, _vp, _vp]),
@@ -272,6 +277,51 @@ def chunk_upsample_noalloc(G, H, idx, idx_offsets, W_bin, *, rows: int, T: int, 
                                       nbins, int(mode), _ptr(S), _ptr(dev_status), _stream(stream))
     _check("chunk_upsample_noalloc", rc)
     return S
+
+
+def chunk_upsample_backward_workspace(rows: int, N: int, nbins: int, d_l: int) -> int:
+    return int(lib().chunk_upsample_backward_workspace(rows, N, nbins, d_l))
+
+
+def chunk_upsample_backward(dS, G, idx, idx_offsets, W_bin, *, rows: int, T: int, offsets=None,
+                            mode: int = BIN_OFFSET, dG=None, dW=None, dH=None, residual: bool = True,
+                            workspace=None, dev_status=None, stream=None):
+    """Gradients of S = h + g_c W_b: (dG fp32 [K, d_g], dW fp32 [nbins, d_g, d_l], dH fp32 [N, d_l] = dS or
+    None when residual is False)."""
+    torch = _torch()
+    _require_cuda(dS, G, idx, idx_offsets, W_bin, offsets)
+    dS2 = dS.reshape(-1, dS.shape[-1]).contiguous()
+    if dS2.dtype != torch.float32:
+        raise TypeError("dS must be float32")
+    N, d_l = dS2.shape
+    nbins, d_g, _ = W_bin.shape
+    K = G.shape[0]
+    dev = dS.device
+    if dG is None:
+        dG = torch.empty(K, d_g, dtype=torch.float32, device=dev)
+    if dW is None:
+        dW = torch.empty(nbins, d_g, d_l, dtype=torch.float32, device=dev)
+    if residual and dH is None:
+        dH = torch.empty(N, d_l, dtype=torch.float32, device=dev)
+    ws = _workspace(chunk_upsample_backward_workspace(rows, N, nbins, d_l), dev, workspace)
+    rc = lib().chunk_upsample_backward(_ptr(dS2), _ptr(G.contiguous()), d_g, _ptr(offsets), T, N, d_l, _ptr(idx),
+                                       _ptr(idx_offsets), rows, K, _ptr(W_bin.contiguous()), nbins, int(mode),
+                                       _ptr(dG), _ptr(dW), _ptr(dH if residual else None), _ptr(ws), ws.numel(),
+                                       _ptr(dev_status), _stream(stream))
+    _check("chunk_upsample_backward", rc)
+    return dG, dW, (dH if residual else None)
+
+
+def chunk_gather_backward(dZ, idx, idx_offsets, *, rows: int, T: int, dH, offsets=None, accumulate: bool = True,
+                          dev_status=None, stream=None):
+    """dH[row start + s_k] (+)= dZ_k in place; returns dH."""
+    _require_cuda(dZ, idx, idx_offsets, dH, offsets)
+    dZ = dZ.contiguous()
+    K, d = dZ.shape
+    rc = lib().chunk_gather_backward(_ptr(dZ), d, _ptr(offsets), T, _ptr(idx), _ptr(idx_offsets), rows, K,
+                                     _ptr(dH), int(bool(accumulate)), _ptr(dev_status), _stream(stream))
+    _check("chunk_gather_backward", rc)
+    return dH
 
 
 def hnet_route_workspace(rows: int, N: int, d: int) -> int:

@@ -44,28 +44,28 @@ struct TmemChol {
 };
 
 // Rank-16 update and shift of the live panel columns of one row:
-// v[p] <- v[16 + p] - sum_c a[c] L(p)[c] for p in [0, P), with L(p) the solved
-// sub-panel row of panel column (kb + 16 + p) in shared memory (stride 20).
-// Columns p > plim are only shifted (a row of the diagonal block in the L role
-// must not touch its upper part, which carries B in the factor mode).
+// v[p] <- v[16 + p] - sum_c a[c] L[kb+16+p][kb+c] for p in [0, P), with the
+// solved sub-panel stored column-major in shared memory (sLT[c * 64 + p]).
+// The loop runs column-outer so the P updates of one step are independent.
+// Entries p >= zfrom are set to zero instead: the part right of the diagonal
+// of a panel row in the L role, which in the factor mode carries B and is
+// still zero there.
 template <int P>
-__device__ __forceinline__ void rank16_shift(float (&v)[64], const float (&a)[16], const float *sL, int plim) {
+__device__ __forceinline__ void rank16_shift(float (&v)[64], const float (&a)[16], const float *sLT, int zfrom) {
 #pragma unroll
-    for (int p = 0; p < P; ++p) {
-        float x = v[16 + p];
-        if (p <= plim) {
-            const float4 *lr = reinterpret_cast<const float4 *>(sL + p * 20);
+    for (int c = 0; c < 16; ++c) {
+        const float4 *lr = reinterpret_cast<const float4 *>(sLT + c * 64);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 l = lr[q];
-                x = fmaf(-a[4 * q], l.x, x);
-                x = fmaf(-a[4 * q + 1], l.y, x);
-                x = fmaf(-a[4 * q + 2], l.z, x);
-                x = fmaf(-a[4 * q + 3], l.w, x);
-            }
+        for (int p4 = 0; p4 < P / 4; ++p4) {
+            const float4 l = lr[p4];
+            v[16 + 4 * p4 + 0] = fmaf(-a[c], l.x, v[16 + 4 * p4 + 0]);
+            v[16 + 4 * p4 + 1] = fmaf(-a[c], l.y, v[16 + 4 * p4 + 1]);
+            v[16 + 4 * p4 + 2] = fmaf(-a[c], l.z, v[16 + 4 * p4 + 2]);
+            v[16 + 4 * p4 + 3] = fmaf(-a[c], l.w, v[16 + 4 * p4 + 3]);
         }
-        v[p] = x;
     }
+#pragma unroll
+    for (int p = 0; p < P; ++p) v[p] = p >= zfrom ? 0.f : v[16 + p];
 }
 
 // Six piece products of a three-way split (dropped terms are below 2^-24):
@@ -144,15 +144,15 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[2];
     __shared__ uint32_t tmem_base;
-    __shared__ __align__(16) float s_L[64][20];     // solved sub-panel rows of the panel's rows (rank-16 update)
-    __shared__ __align__(16) float s_Ld[16][20];    // factored 16 x 16 diagonal block
-    __shared__ float s_rl[16];                      // 1 / L_kk of the diagonal block
+    __shared__ __align__(16) float s_LT[16][64];    // solved sub-panel of the panel's rows, column-major
+    __shared__ __align__(16) float s_LdT[16][16];   // factored 16 x 16 diagonal block, column-major
+    __shared__ __align__(16) float s_rl[16];        // 1 / L_kk of the diagonal block
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int blk = warp >> 2, lb = (warp & 3) * 32;
     const int row = blk * 128 + lb + lane;
     const uint32_t region = (tc::smem_u32(smraw) + 1023u) & ~1023u;
     float *done = reinterpret_cast<float *>(smraw + (region - tc::smem_u32(smraw)) + TmemChol::REGION);
-    for (int e = tid; e < 64 * 20; e += TmemChol::NT) (&s_L[0][0])[e] = 0.f;
+    for (int e = tid; e < 16 * 64; e += TmemChol::NT) (&s_LT[0][0])[e] = 0.f;
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
         tc::mbar_init(&mbar[0], 1);
@@ -288,68 +288,83 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 const bool diag = ii >= 0 && ii < 16;
                 float a[16];
                 if (diag) {
+                    // branch-free (selects only): the half-warp stays converged for its shuffles,
+                    // and the per-pivot work on the serial path is one broadcast, one rsqrt and
+                    // one fma; each lane keeps its own pivot's values and writes them afterwards
                     const int lb0 = lane & 16;
                     const unsigned mask = 0xFFFFu << lb0;
+                    float rl_mine = 1.f, e_mine = 0.f;
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float e = __shfl_sync(mask, v[c], lb0 + c);
+                        const float e = __shfl_sync(mask, v[c], lb0 + c);   // excess of column c
                         const float rlc = rsqrtf(1.f + e);
-                        if (ii == c) {
-                            v[c] = (1.f + e) * rlc;                       // L_cc
-                            s_rl[c] = rlc;
-                            if (!FACTOR && kb + c < nb) dR[start + j0 + kb + c] = 0.5f * log1pf(e);
-                        } else if (ii > c) {
-                            v[c] *= rlc;                                  // L_ii,c
-                        }
+                        const float li = v[c] * rlc;                        // L_ii,c for ii > c
 #pragma unroll
                         for (int c2 = 0; c2 < 16; ++c2) {
                             if (c2 > c) {
-                                const float l2 = __shfl_sync(mask, v[c], lb0 + c2);
-                                if (ii >= c2) v[c2] = fmaf(-v[c], l2, v[c2]);
+                                const float w = __shfl_sync(mask, v[c], lb0 + c2);
+                                const float u = fmaf(-li, w * rlc, v[c2]);
+                                v[c2] = ii >= c2 ? u : v[c2];
                             }
                         }
+                        const bool piv = ii == c;
+                        v[c] = piv ? (1.f + e) * rlc : (ii > c ? li : v[c]);  // L_cc on the pivot row
+                        rl_mine = piv ? rlc : rl_mine;
+                        e_mine = piv ? e : e_mine;
                     }
+                    s_rl[ii] = rl_mine;
+                    if (!FACTOR && kb + ii < nb) dR[start + j0 + kb + ii] = 0.5f * log1pf(e_mine);
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const float x = c <= ii ? v[c] : 0.f;
-                        s_Ld[ii][c] = x;
+                        s_LdT[c][ii] = x;
                         if (c <= ii) done[row * 65 + kb + c] = x;
                     }
                 }
                 __syncthreads();
                 const bool live = FACTOR || ii >= 16;        // INSEG rows at or above the block are done
                 if (live) {
+                    // right-looking solve against the diagonal block: a[m] is final once the
+                    // columns before m are applied; a diagonal-block row takes the B role
+                    // (B_im = 0 for m < ii, B_ii = 1/L_ii)
+                    float rl[16];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        if (diag && c <= ii) {
-                            a[c] = c == ii ? s_rl[c] : 0.f;         // B role of a diagonal-block row: B_ii = 1/L_ii
-                        } else {
-                            const float4 *lr = reinterpret_cast<const float4 *>(&s_Ld[c][0]);
-                            float x = v[c];
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 r4 = reinterpret_cast<const float4 *>(s_rl)[j];
+                        rl[4 * j] = r4.x; rl[4 * j + 1] = r4.y; rl[4 * j + 2] = r4.z; rl[4 * j + 3] = r4.w;
+                    }
 #pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                const float4 l = lr[q4];
-                                if (4 * q4 + 0 < c) x = fmaf(-a[4 * q4 + 0], l.x, x);
-                                if (4 * q4 + 1 < c) x = fmaf(-a[4 * q4 + 1], l.y, x);
-                                if (4 * q4 + 2 < c) x = fmaf(-a[4 * q4 + 2], l.z, x);
-                                if (4 * q4 + 3 < c) x = fmaf(-a[4 * q4 + 3], l.w, x);
+                    for (int m = 0; m < 16; ++m) {
+                        float am = v[m] * rl[m];
+                        if (diag && m <= ii) am = m == ii ? rl[m] : 0.f;
+                        a[m] = am;
+                        const float4 *lr = reinterpret_cast<const float4 *>(&s_LdT[m][0]);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if (4 * j + 3 > m) {
+                                const float4 l = lr[j];
+                                if (4 * j + 0 > m) v[4 * j + 0] = fmaf(-am, l.x, v[4 * j + 0]);
+                                if (4 * j + 1 > m) v[4 * j + 1] = fmaf(-am, l.y, v[4 * j + 1]);
+                                if (4 * j + 2 > m) v[4 * j + 2] = fmaf(-am, l.z, v[4 * j + 2]);
+                                v[4 * j + 3] = fmaf(-am, l.w, v[4 * j + 3]);
                             }
-                            a[c] = x * s_rl[c];
-                            done[row * 65 + kb + c] = a[c];
                         }
                     }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (!(diag && c <= ii)) done[row * 65 + kb + c] = a[c];
                     if (ii >= 16 && rel < 64) {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) s_L[rel][c] = a[c];
+                        for (int c = 0; c < 16; ++c) s_LT[c][rel] = a[c];
                     }
                 }
                 __syncthreads();
                 if (live && q + 1 < nsub) {
-                    const float *sL = &s_L[kb + 16][0];
-                    const int plim = (FACTOR && ii >= 16 && rel < 64) ? ii - 16 : 64;
-                    if (q == 0) rank16_shift<48>(v, a, sL, plim);
-                    else if (q == 1) rank16_shift<32>(v, a, sL, plim);
-                    else rank16_shift<16>(v, a, sL, plim);
+                    const float *sLT = &s_LT[0][kb + 16];
+                    const int zfrom = (FACTOR && ii >= 16 && rel < 64) ? ii - 15 : 64;
+                    if (q == 0) rank16_shift<48>(v, a, sLT, zfrom);
+                    else if (q == 1) rank16_shift<32>(v, a, sLT, zfrom);
+                    else rank16_shift<16>(v, a, sLT, zfrom);
                 }
             }
 #pragma unroll

@@ -9,6 +9,7 @@
 // each bin's positions are contiguous; the product is then a grouped GEMM over
 // bins on tcgen05 whose A rows are gathered chunk vectors and whose output rows
 // are scattered back to their positions with the residual added.
+#include "bins.cuh"
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -51,42 +52,10 @@ __global__ void __launch_bounds__(256) classify_kernel(const int64_t *offsets, i
     __syncthreads();
     for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < N;
          p += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = offsets ? find_row(offsets, rows, p) : p / T;
-        int64_t a, n;
-        row_bounds(offsets, r, T, a, n);
-        const int64_t t = p - a;
-        const int64_t ia = idx_offsets[r];
-        const int64_t kr = idx_offsets[r + 1] - ia;
-        int64_t c = 0;
-        if (kr <= 0 || idx[ia] != 0) {
-            flag(st, DBC_ERR_BOUNDS);
-        } else {
-            int64_t lo = 0, hi = kr;     // idx[ia+lo] <= t < idx[ia+hi] (hi = kr: +inf)
-            while (hi - lo > 1) {
-                const int64_t mid = (lo + hi) >> 1;
-                if (idx[ia + mid] <= t) lo = mid; else hi = mid;
-            }
-            c = lo;
-        }
-        const int64_t sc = kr > 0 ? idx[ia + c] : 0;
-        int64_t b;
-        if (mode == DBC_BIN_IN_CHUNK_OFFSET) {
-            b = t - sc;
-            if (b > nbins - 1) b = nbins - 1;
-        } else if (mode == DBC_BIN_IN_CHUNK_FRACTION) {
-            const int64_t nxt = (c + 1 < kr) ? idx[ia + c + 1] : n;
-            const int64_t len = nxt - sc;
-            b = len > 0 ? ((int64_t)nbins * (t - sc)) / len : 0;
-        } else {
-            b = ((int64_t)t * nbins) / n;
-        }
-        if (b < 0 || b >= nbins) {
-            flag(st, DBC_ERR_BOUNDS);
-            b = b < 0 ? 0 : nbins - 1;
-        }
-        L.chunk[p] = (int32_t)(ia + c);
-        L.bin[p] = (uint8_t)b;
-        atomicAdd(&h[b], 1);
+        const PosClass pc = classify_position(p, offsets, T, idx, idx_offsets, rows, nbins, mode, st);
+        L.chunk[p] = pc.chunk;
+        L.bin[p] = (uint8_t)pc.bin;
+        atomicAdd(&h[pc.bin], 1);
     }
     __syncthreads();
     for (int b = threadIdx.x; b < nbins; b += blockDim.x)

@@ -173,6 +173,59 @@ DBC_API dbc_status chunk_upsample(const void *G, int64_t d_g, const void *H, int
                           dbc_stream_t stream);
 
 /* -------------------------------------------------------------------------
+ * chunk_upsample_backward -- gradients of the upsampling (for training).
+ *
+ * ByteFlow (summary stage 4; notes "Key design 4"), differentiated: with
+ * dS = dL/dS for S_t = h_t + g_{c(t)} W_{b(t)},
+ *   dG_k = sum over t in chunk k of dS_t W_{b(t)}^T,
+ *   dW_b = sum over t in bin b of g_{c(t)}^T dS_t   (summed over all rows),
+ *   dH_t = dS_t (the residual; the gather adds dG at the boundaries, see
+ *          chunk_gather_backward).
+ * The Top-K selection itself passes no gradient (notes "Key design 2").
+ *
+ * dS       fp32 [N, d_l] upstream gradient; offsets NULL (dense) or int64 [rows+1].
+ * G        bf16 [total_K, d_g] the chunk vectors of the forward call.
+ * idx, idx_offsets, W_bin, nbins, mode: as in chunk_upsample.
+ * dG       out fp32 [total_K, d_g]; dW out fp32 [nbins, d_g, d_l] (both
+ *          overwritten, zeroed by the call itself).
+ * dH       out fp32 [N, d_l] = dS, or NULL to skip the copy.
+ * ws       workspace of chunk_upsample_backward_workspace(rows, N, nbins, d_l)
+ *          bytes (about 4 d_l + 26 bytes per position).
+ * All pointers 16-byte aligned.  Supported: d_g a multiple of 128, d_l a
+ * multiple of 64, both up to 4096.  dG and dW are sums of fp32 partial
+ * results added with atomics: repeated calls agree to rounding, not bitwise.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA; device flags BOUNDS,
+ * TIMEOUT.
+ * ------------------------------------------------------------------------- */
+DBC_API size_t chunk_upsample_backward_workspace(int64_t rows, int64_t N, int nbins, int64_t d_l);
+DBC_API dbc_status chunk_upsample_backward(const float *dS, const void *G, int64_t d_g,
+                                           const int64_t *offsets, int64_t T, int64_t N, int64_t d_l,
+                                           const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
+                                           int64_t total_K, const void *W_bin, int nbins, int mode,
+                                           float *dG, float *dW, float *dH, void *ws, size_t ws_bytes,
+                                           int32_t *dev_status, dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * chunk_gather_backward -- adjoint of chunk_gather's copy.
+ *
+ * ByteFlow (summary stage 2): z_k = h_{s_k}, so dL/dh_{s_k} receives dL/dz_k
+ * and every other position nothing:
+ *   dH[row start + s_k] = dZ_k          (accumulate == 0), or
+ *   dH[row start + s_k] += dZ_k         (accumulate != 0, e.g. onto the
+ *                                        residual dH of chunk_upsample_backward).
+ * Rows of dH that are no boundary are left untouched.
+ *
+ * dZ       fp32 [total_K, d]; dH in/out fp32 [N, d]; idx, idx_offsets,
+ *          offsets as in chunk_gather.  d a multiple of 4; 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA; device flag BOUNDS (a boundary
+ * outside its row is skipped).
+ * ------------------------------------------------------------------------- */
+DBC_API dbc_status chunk_gather_backward(const float *dZ, int64_t d, const int64_t *offsets, int64_t T,
+                                         const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
+                                         int64_t total_K, float *dH, int accumulate, int32_t *dev_status,
+                                         dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
  * chunk_upsample_noalloc -- chunk_upsample for callers that cannot allocate.
  *
  * No passage of the pages corresponds to this entry point; it is a deployment

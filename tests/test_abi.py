@@ -74,3 +74,23 @@ def test_argument_errors_return_before_launch(L):
     u = L.chunk_upsample
     assert u(None, 64, None, 1, None, 8, 8, 64, None, None, 1, None, 0, 0, None, None, 0, None, None) == 1
     assert u(None, 64, None, 1, None, 8, 8, 64, None, None, 1, None, 16, 7, None, None, 0, None, None) == 1
+
+
+def test_backward_argument_errors_return_before_launch(L):
+    ub = L.chunk_upsample_backward
+    # d_g not a multiple of 128
+    assert ub(None, None, 64, None, 8, 8, 64, None, None, 1, 2, None, 16, 0, None, None, None, None, 0, None,
+              None) == 2
+    # nbins out of range
+    assert ub(None, None, 128, None, 8, 8, 64, None, None, 1, 2, None, 0, 0, None, None, None, None, 0, None,
+              None) == 1
+    # missing outputs
+    assert ub(None, None, 128, None, 8, 8, 64, None, None, 1, 2, None, 16, 0, None, None, None, None, 0, None,
+              None) == 1
+    gb = L.chunk_gather_backward
+    # d not a multiple of 4
+    assert gb(None, 6, None, 8, None, None, 1, 2, None, 1, None, None) == 2
+    # nothing to do
+    assert gb(None, 8, None, 8, None, None, 1, 0, None, 1, None, None) == 0
+    import dynamic_byte_chunking_b200 as dbc
+    assert dbc.chunk_upsample_backward_workspace(8, 65536, 16, 256) >= 2 * 65536 * 256 * 2
