@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--rows", action="store_true",
                     help="time every hot-path row on its own workload family (one JSON line per row)")
     ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--families", default="tiny,byteflow,bytegen,wide,ragged",
+                    help="workload families measured by --rows (comma-separated)")
     ap.add_argument("--traffic-from", default=None, metavar="CSV",
                     help="convert an ncu --csv launch list with dram__bytes_read.sum and dram__bytes_write.sum "
                          "(taken on this workload) into profiles/dram_traffic_byteflow.json, then exit")
@@ -277,7 +279,7 @@ def run_rows(args):
         line = {"row": row, "workload": fam, "ms": ms, **kv, "peak_source": src}
         print(json.dumps(line), flush=True)
 
-    for fam in ["tiny", "byteflow", "bytegen", "wide", "ragged"]:
+    for fam in [f for f in args.families.split(",") if f]:
         w = workloads.make(fam)
         H = bf(w.H_bits) if w.dtype == "bf16" else torch.from_numpy(w.H_bits).to(dev)
         offs = torch.from_numpy(w.offsets).to(dev)

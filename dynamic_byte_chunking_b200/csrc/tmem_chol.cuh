@@ -383,18 +383,9 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     if (k >= nb) v[k] = 0.f;
             }
             if (FACTOR) {
-                // B panel (rows >= j1 are zero there) -> global; operand rows -> smem
-                __nv_bfloat16 *g = Bs + (size_t)row * D + j0;
-                if (row < j1) {
-                    stage_row(region, row, v, g, (size_t)D * D);
-                } else {
-                    stage_row(region, row, v, nullptr, 0);
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-                    for (int p = 0; p < 3; ++p)
-#pragma unroll
-                        for (int k8 = 0; k8 < 8; ++k8) *reinterpret_cast<uint4 *>(g + (size_t)p * D * D + k8 * 8) = z;
-                }
+                // B panel -> global (rows >= j1 are zero in these columns and are never stored: the
+                // product B B^T below zero-fills them); operand rows -> smem
+                stage_row(region, row, v, row < j1 ? Bs + (size_t)row * D + j0 : nullptr, (size_t)D * D);
             } else if (j1 < n) {
                 stage_row(region, row, v, nullptr, 0);
             }
@@ -465,27 +456,42 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 if (!ok) break;
             }
             if (!ok) break;
-            __nv_bfloat16 *A = A3 + (size_t)s * 3 * D * D + (size_t)row * D;
+            // A -> three bf16 pieces, staged per 64-column block in shared memory (row-major, 144-byte
+            // rows) and written out as whole 128-byte row segments
+            __nv_bfloat16 *Ag = A3 + (size_t)s * 3 * D * D;
+            uint8_t *stg = smraw + (region - tc::smem_u32(smraw));
+            constexpr int RS = 144;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float t16[16];
-                tc::tmem_ld16(trow + (uint32_t)c0, t16);
-                uint32_t hh[8], mm[8], ll[8];
+            for (int cb = 0; cb < D; cb += 64) {
+#pragma unroll 1
+                for (int j = 0; j < 4; ++j) {
+                    float t16[16];
+                    tc::tmem_ld16(trow + (uint32_t)(cb + 16 * j), t16);
+                    uint32_t hh[8], mm[8], ll[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint16_t h0, m0, l0, h1, m1, l1;
-                    split3v(t16[2 * q], h0, m0, l0);
-                    split3v(t16[2 * q + 1], h1, m1, l1);
-                    hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                    mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
-                    ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                    for (int q = 0; q < 8; ++q) {
+                        uint16_t h0, m0, l0, h1, m1, l1;
+                        split3v(t16[2 * q], h0, m0, l0);
+                        split3v(t16[2 * q + 1], h1, m1, l1);
+                        hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                        mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
+                        ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                    }
+                    uint4 *d0 = reinterpret_cast<uint4 *>(stg + (size_t)row * RS + j * 32);
+                    uint4 *d1 = reinterpret_cast<uint4 *>(stg + (size_t)(256 + row) * RS + j * 32);
+                    uint4 *d2 = reinterpret_cast<uint4 *>(stg + (size_t)(512 + row) * RS + j * 32);
+                    d0[0] = make_uint4(hh[0], hh[1], hh[2], hh[3]); d0[1] = make_uint4(hh[4], hh[5], hh[6], hh[7]);
+                    d1[0] = make_uint4(mm[0], mm[1], mm[2], mm[3]); d1[1] = make_uint4(mm[4], mm[5], mm[6], mm[7]);
+                    d2[0] = make_uint4(ll[0], ll[1], ll[2], ll[3]); d2[1] = make_uint4(ll[4], ll[5], ll[6], ll[7]);
                 }
-                uint4 *d0 = reinterpret_cast<uint4 *>(A + c0);
-                uint4 *d1 = reinterpret_cast<uint4 *>(A + (size_t)D * D + c0);
-                uint4 *d2 = reinterpret_cast<uint4 *>(A + (size_t)2 * D * D + c0);
-                d0[0] = make_uint4(hh[0], hh[1], hh[2], hh[3]); d0[1] = make_uint4(hh[4], hh[5], hh[6], hh[7]);
-                d1[0] = make_uint4(mm[0], mm[1], mm[2], mm[3]); d1[1] = make_uint4(mm[4], mm[5], mm[6], mm[7]);
-                d2[0] = make_uint4(ll[0], ll[1], ll[2], ll[3]); d2[1] = make_uint4(ll[4], ll[5], ll[6], ll[7]);
+                __syncthreads();
+                for (int e = tid; e < 3 * 256 * 8; e += TmemChol::NT) {
+                    const int pr = e >> 3, ch = e & 7;                 // piece-row (piece * 256 + row), chunk
+                    const uint4 x = *reinterpret_cast<const uint4 *>(stg + (size_t)pr * RS + ch * 16);
+                    const int pc = pr >> 8, r = pr & 255;
+                    *reinterpret_cast<uint4 *>(Ag + (size_t)pc * D * D + (size_t)r * D + cb + ch * 8) = x;
+                }
+                __syncthreads();
             }
             tc::fence_before_sync();
             __syncthreads();

@@ -108,7 +108,10 @@ struct BinTC {
     static constexpr uint32_t A_BYTES = 128 * 128;
     static constexpr uint32_t B_BYTES = 4 * 64 * 128;          // up to 256 columns x 64 K, MN-major
     static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
-    static constexpr size_t SMEM = NS * STAGE + 1024;
+    static constexpr uint32_t HBUF = 128 * 256 * 2;             // the tile's residual rows (bf16 H)
+    // bf16 H is prefetched into shared memory while the MMAs run; fp32 H is read in the epilogue
+    template <class IN>
+    static constexpr size_t smem() { return NS * STAGE + (sizeof(IN) == 2 ? HBUF : 0) + 1024; }
 };
 
 template <class IN>
@@ -161,10 +164,23 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
         }
     };
     const uint32_t idesc = tc::idesc_bf16(128, nt, false, true);
+    constexpr bool kPrefetchH = sizeof(IN) == 2;
+    const uint32_t hbuf = base + BinTC::NS * BinTC::STAGE;
     bool ok = true;
     for (int c = 0; c < BinTC::NS - 1; ++c) {
         if (c < nchunks) load(c, base + (uint32_t)c * BinTC::STAGE);
         tc::cp_async_commit();
+        if (kPrefetchH && c == 0) {
+            // residual rows of this tile: [128][nt] bf16, row-major (zeros for empty rows)
+            const int nc = nt / 8;
+            for (int e = tid; e < 128 * nc; e += 128) {
+                const int r = e / nc, ch = e - (e / nc) * nc;
+                const int p = pos[r];
+                const IN *src = H + (size_t)(p >= 0 ? p : 0) * dl + n0 + ch * 8;
+                tc::cp_async16(hbuf + (uint32_t)(r * nt + ch * 8) * 2, src, p >= 0 ? 16u : 0u);
+            }
+            tc::cp_async_commit();
+        }
     }
     for (int c = 0; c < nchunks; ++c) {
         const int cn = c + BinTC::NS - 1;
@@ -217,8 +233,9 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
                 const float4 a1 = *reinterpret_cast<const float4 *>(t + 4);
                 float h[8];
                 const IN *hrow = H + (size_t)p * dl + n0 + c8 * 8;
-                if (sizeof(IN) == 2) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(hrow);
+                if (kPrefetchH) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(smraw + (hbuf - tc::smem_u32(smraw)) +
+                                                                     (size_t)(rr * nt + c8 * 8) * 2);
                     const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) h[i] = __bfloat162float(hb[i]);
@@ -253,14 +270,14 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
     dim3 g((unsigned)((N + 127) / 128 + nbins), (unsigned)((d_l + 255) / 256));
     if (dtype == DBC_BF16) {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)BinTC::SMEM);
-        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 128, BinTC::SMEM, s>>>(
+                             (int)BinTC::smem<__nv_bfloat16>());
+        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 128, BinTC::smem<__nv_bfloat16>(), s>>>(
             static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
             static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
     } else {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)BinTC::SMEM);
-        bin_gemm_tc_kernel<float><<<g, 128, BinTC::SMEM, s>>>(
+                             (int)BinTC::smem<float>());
+        bin_gemm_tc_kernel<float><<<g, 128, BinTC::smem<float>(), s>>>(
             static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
             static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
     }

@@ -29,6 +29,8 @@ namespace ub {
 constexpr int kMaxBins = 64;
 constexpr int kBlk = 256;       // positions per block of the run scan
 constexpr int kSplit = 512;     // products per CTA of the weight-gradient GEMM
+constexpr int kLong = 64;       // runs longer than this are summed by whole CTAs, kTile positions at a time
+constexpr int kTile = 256;
 
 struct Layout {
     int32_t *chunk;       // [N] chunk of each position
@@ -45,6 +47,9 @@ struct Layout {
     int32_t *tile_start;  // [kMaxBins + 1] first 128-slot tile of each bin
     int32_t *split_start; // [kMaxBins + 1] first kSplit-slot split of each bin
     int32_t *nprod;       // [1] number of products P
+    int32_t *long_pid;    // [N / (kLong + 1) + 1] products whose run is longer than kLong
+    int32_t *nlong;       // [1]
+    float *Dlong;         // [N / (kLong + 1) + 1][d_l] fp32 sums of the long runs
     __nv_bfloat16 *Dh;    // [N][d_l] per slot: sum of dS over the product's run, high bf16 piece
     __nv_bfloat16 *Dl;    // [N][d_l] low piece
     size_t bytes;
@@ -68,6 +73,10 @@ inline Layout carve(void *ws, int64_t N, int64_t d_l) {
     L.tile_start = c.take<int32_t>(kMaxBins + 1);
     L.split_start = c.take<int32_t>(kMaxBins + 1);
     L.nprod = c.take<int32_t>(1);
+    const int64_t maxlong = N / (kLong + 1) + 1;
+    L.long_pid = c.take<int32_t>(maxlong);
+    L.nlong = c.take<int32_t>(1);
+    L.Dlong = c.take<float>((size_t)maxlong * d_l);
     L.Dh = c.take<__nv_bfloat16>((size_t)N * d_l);
     L.Dl = c.take<__nv_bfloat16>((size_t)N * d_l);
     L.bytes = c.off;
@@ -178,6 +187,7 @@ __global__ void scan_bins_kernel(int nbins, Layout L) {
         L.bin_start[nbins] = s;
         L.tile_start[nbins] = t;
         L.split_start[nbins] = q;
+        *L.nlong = 0;
     }
 }
 
@@ -212,8 +222,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
 }
 
-// One warp per product: D = sum of its dS rows (in position order), stored as
-// hi + lo bf16 pieces at the product's slot; optionally dH = dS on the way.
+__device__ __forceinline__ void store_pieces(__nv_bfloat16 *Dh, __nv_bfloat16 *Dl, int64_t off, float4 acc) {
+    const float hx = __bfloat162float(__float2bfloat16_rn(acc.x));
+    const float hy = __bfloat162float(__float2bfloat16_rn(acc.y));
+    const float hz = __bfloat162float(__float2bfloat16_rn(acc.z));
+    const float hw = __bfloat162float(__float2bfloat16_rn(acc.w));
+    *reinterpret_cast<uint2 *>(Dh + off) = make_uint2(pack_bf16x2(hx, hy), pack_bf16x2(hz, hw));
+    *reinterpret_cast<uint2 *>(Dl + off) =
+        make_uint2(pack_bf16x2(acc.x - hx, acc.y - hy), pack_bf16x2(acc.z - hz, acc.w - hw));
+}
+
+__device__ __forceinline__ void add4(float4 &a, const float4 &x) {
+    a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+}
+
+// One warp per product of at most kLong positions: D = sum of its dS rows (in
+// position order, four rows in flight), stored as hi + lo bf16 pieces at the
+// product's slot; optionally dH = dS on the way.  Longer products are queued
+// for long_sum_kernel (their fp32 sum row is cleared here).
 __global__ void __launch_bounds__(256) sum_kernel(const float4 *__restrict__ dS, int64_t nv4, float4 *dH,
                                                   Layout L) {
     const int lane = threadIdx.x & 31;
@@ -221,23 +247,100 @@ __global__ void __launch_bounds__(256) sum_kernel(const float4 *__restrict__ dS,
     const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t pid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pid < P; pid += nw) {
         const int64_t a = L.t0[pid], e = L.t0[pid + 1];
+        if (e - a > kLong) {
+            int j = 0;
+            if (lane == 0) {
+                j = atomicAdd(L.nlong, 1);
+                L.long_pid[j] = (int32_t)pid;
+            }
+            j = __shfl_sync(0xffffffffu, j, 0);
+            float4 *row = reinterpret_cast<float4 *>(L.Dlong + (size_t)j * nv4 * 4);
+            for (int64_t f = lane; f < nv4; f += 32) row[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+            continue;
+        }
         const int64_t s = L.slot[pid];
-        uint2 *hi = reinterpret_cast<uint2 *>(L.Dh + s * nv4 * 4);
-        uint2 *lo = reinterpret_cast<uint2 *>(L.Dl + s * nv4 * 4);
         for (int64_t f = lane; f < nv4; f += 32) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int64_t t = a; t < e; ++t) {
+            int64_t t = a;
+            for (; t + 4 <= e; t += 4) {
+                const float4 x0 = dS[t * nv4 + f], x1 = dS[(t + 1) * nv4 + f];
+                const float4 x2 = dS[(t + 2) * nv4 + f], x3 = dS[(t + 3) * nv4 + f];
+                add4(acc, x0); add4(acc, x1); add4(acc, x2); add4(acc, x3);
+                if (dH) {
+                    dH[t * nv4 + f] = x0; dH[(t + 1) * nv4 + f] = x1;
+                    dH[(t + 2) * nv4 + f] = x2; dH[(t + 3) * nv4 + f] = x3;
+                }
+            }
+            for (; t < e; ++t) {
                 const float4 x = dS[t * nv4 + f];
-                acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+                add4(acc, x);
                 if (dH) dH[t * nv4 + f] = x;
             }
-            const float hx = __bfloat162float(__float2bfloat16_rn(acc.x));
-            const float hy = __bfloat162float(__float2bfloat16_rn(acc.y));
-            const float hz = __bfloat162float(__float2bfloat16_rn(acc.z));
-            const float hw = __bfloat162float(__float2bfloat16_rn(acc.w));
-            hi[f] = make_uint2(pack_bf16x2(hx, hy), pack_bf16x2(hz, hw));
-            lo[f] = make_uint2(pack_bf16x2(acc.x - hx, acc.y - hy), pack_bf16x2(acc.z - hz, acc.w - hw));
+            store_pieces(L.Dh, L.Dl, (s * nv4 + f) * 4, acc);
         }
+    }
+}
+
+// Long products, split into kTile-position tiles dealt round-robin over the
+// CTAs: 4 position groups x 64 float4 columns per pass, partial sums combined
+// in shared memory and added into the product's fp32 row.
+__global__ void __launch_bounds__(256) long_sum_kernel(const float4 *__restrict__ dS, int64_t nv4, float4 *dH,
+                                                       Layout L) {
+    __shared__ float4 part[4][64];
+    const int tid = threadIdx.x, pg = tid >> 6, fl = tid & 63;
+    const int nl = *L.nlong;
+    const int64_t G = gridDim.x;
+    int64_t tile_base = 0;
+    for (int j = 0; j < nl; ++j) {
+        const int64_t pid = L.long_pid[j];
+        const int64_t a = L.t0[pid], e = L.t0[pid + 1];
+        const int64_t ntile = (e - a + kTile - 1) / kTile;
+        const int64_t i0 = ((int64_t)blockIdx.x - tile_base % G + G) % G;
+        for (int64_t i = i0; i < ntile; i += G) {
+            const int64_t p0 = a + i * kTile, p1 = p0 + kTile < e ? p0 + kTile : e;
+            for (int64_t fb = 0; fb < nv4; fb += 64) {
+                const int64_t f = fb + fl;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (f < nv4) {
+                    int64_t t = p0 + pg;
+                    for (; t + 12 < p1; t += 16) {
+                        const float4 x0 = dS[t * nv4 + f], x1 = dS[(t + 4) * nv4 + f];
+                        const float4 x2 = dS[(t + 8) * nv4 + f], x3 = dS[(t + 12) * nv4 + f];
+                        add4(acc, x0); add4(acc, x1); add4(acc, x2); add4(acc, x3);
+                        if (dH) {
+                            dH[t * nv4 + f] = x0; dH[(t + 4) * nv4 + f] = x1;
+                            dH[(t + 8) * nv4 + f] = x2; dH[(t + 12) * nv4 + f] = x3;
+                        }
+                    }
+                    for (; t < p1; t += 4) {
+                        const float4 x = dS[t * nv4 + f];
+                        add4(acc, x);
+                        if (dH) dH[t * nv4 + f] = x;
+                    }
+                }
+                part[pg][fl] = acc;
+                __syncthreads();
+                if (pg == 0 && f < nv4) {
+                    float4 r = part[0][fl];
+                    add4(r, part[1][fl]); add4(r, part[2][fl]); add4(r, part[3][fl]);
+                    atomicAdd(reinterpret_cast<float4 *>(L.Dlong + (size_t)j * nv4 * 4) + f, r);
+                }
+                __syncthreads();
+            }
+        }
+        tile_base += ntile;
+    }
+}
+
+// One warp per long product: its fp32 sum -> hi + lo pieces at its slot.
+__global__ void __launch_bounds__(256) long_final_kernel(int64_t nv4, Layout L) {
+    const int lane = threadIdx.x & 31;
+    const int nl = *L.nlong;
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); j < nl; j += nw) {
+        const int64_t s = L.slot[L.long_pid[j]];
+        const float4 *row = reinterpret_cast<const float4 *>(L.Dlong + (size_t)j * nv4 * 4);
+        for (int64_t f = lane; f < nv4; f += 32) store_pieces(L.Dh, L.Dl, (s * nv4 + f) * 4, row[f]);
     }
 }
 
@@ -581,6 +684,9 @@ extern "C" dbc_status chunk_upsample_backward(const float *dS, const void *G, in
     const int64_t wgrid = std::max<int64_t>(1, std::min<int64_t>((N + 7) / 8, (int64_t)sms * 16));
     ub::sum_kernel<<<(unsigned)wgrid, 256, 0, s>>>(reinterpret_cast<const float4 *>(dS), d_l / 4,
                                                    reinterpret_cast<float4 *>(dH), L);
+    ub::long_sum_kernel<<<(unsigned)(2 * sms), 256, 0, s>>>(reinterpret_cast<const float4 *>(dS), d_l / 4,
+                                                            reinterpret_cast<float4 *>(dH), L);
+    ub::long_final_kernel<<<(unsigned)sms, 256, 0, s>>>(d_l / 4, L);
     cudaFuncSetAttribute(ub::dg_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ub::DgTC::SMEM);
     dim3 gg((unsigned)((N + 127) / 128 + nbins), (unsigned)((d_g + 255) / 256));
     ub::dg_gemm_kernel<<<gg, 128, ub::DgTC::SMEM, s>>>(static_cast<const __nv_bfloat16 *>(W_bin), d_g, d_l, nbins,
@@ -590,7 +696,7 @@ extern "C" dbc_status chunk_upsample_backward(const float *dS, const void *G, in
             (unsigned)((d_l + 255) / 256));
     ub::dw_gemm_kernel<<<gw, 128, ub::DwTC::SMEM, s>>>(static_cast<const __nv_bfloat16 *>(G), d_g, d_l, nbins, L,
                                                       dW, total_K, dev_status);
-    count_launches(9);
+    count_launches(11);
     return launch_status();
 }
 
