@@ -268,24 +268,39 @@ __global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__re
     };
     const bool ok = tc_gemm_kmajor<D, VCfg<D>::NS>(tbase, 3 * KC, base, mbar, load, st);
     if (ok) {
+        // per 64-column block: TMEM -> three bf16 pieces in shared memory (row-major, 144-byte
+        // rows, reusing the stage buffers) -> whole 128-byte row segments to V3
+        tc::cp_async_wait<0>();
+        __syncthreads();
+        uint8_t *stg = smraw + (base - tc::smem_u32(smraw));
+        constexpr int RS = 144;
         const int row = warp * 32 + lane;
-        const bool valid = row < rows_valid;
-        __nv_bfloat16 *v0 = V3 + (size_t)(start + mb * 128 + row) * D;
+        __nv_bfloat16 *vb = V3 + (size_t)(start + mb * 128) * D;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
-            float v[16];
-            tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-            if (valid) {
+        for (int cb = 0; cb < D; cb += 64) {
+#pragma unroll 1
+            for (int j = 0; j < 4; ++j) {
+                float v[16];
+                tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cb + 16 * j), v);
                 __align__(16) __nv_bfloat16 h[16], m[16], l[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) split3(scale * v[i], h[i], m[i], l[i]);
-                uint4 *d0 = reinterpret_cast<uint4 *>(v0 + c0);
-                uint4 *d1 = reinterpret_cast<uint4 *>(v0 + (size_t)N * D + c0);
-                uint4 *d2 = reinterpret_cast<uint4 *>(v0 + (size_t)2 * N * D + c0);
-                d0[0] = reinterpret_cast<uint4 *>(h)[0]; d0[1] = reinterpret_cast<uint4 *>(h)[1];
-                d1[0] = reinterpret_cast<uint4 *>(m)[0]; d1[1] = reinterpret_cast<uint4 *>(m)[1];
-                d2[0] = reinterpret_cast<uint4 *>(l)[0]; d2[1] = reinterpret_cast<uint4 *>(l)[1];
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(p == 0 ? h : (p == 1 ? m : l));
+                    uint4 *d = reinterpret_cast<uint4 *>(stg + (size_t)(p * 128 + row) * RS + j * 32);
+                    d[0] = src[0];
+                    d[1] = src[1];
+                }
             }
+            __syncthreads();
+            for (int e = tid; e < 3 * 128 * 8; e += 128) {
+                const int pr = e >> 3, ch = e & 7, p = pr >> 7, r = pr & 127;
+                if (r < rows_valid)
+                    *reinterpret_cast<uint4 *>(vb + (size_t)p * N * D + (size_t)r * D + cb + ch * 8) =
+                        *reinterpret_cast<const uint4 *>(stg + (size_t)pr * RS + ch * 16);
+            }
+            __syncthreads();
         }
     }
     tc::fence_before_sync();
