@@ -308,6 +308,129 @@ __global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__re
     if (warp == 0) tc::tmem_dealloc(tbase, D);
 }
 
+// V = c X_s A_s for a whole segment of up to 256 positions in one CTA (d = 256):
+// both 128-row blocks accumulate in TMEM (columns 0 and 256), so each piece of
+// A_s is read once per segment; written as three bf16 pieces through shared
+// memory in whole 128-byte row segments.
+struct VSegCfg {
+    static constexpr int NS = 3;
+    static constexpr uint32_t X_BYTES = 2 * 128 * 128;         // 256 positions x 64 K
+    static constexpr uint32_t STAGE = X_BYTES + 256 * 128;     // + 256 rows of A x 64 K
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+};
+static_assert(VSegCfg::NS * VSegCfg::STAGE >= 3u * 256u * 144u, "epilogue staging must fit in the stages");
+
+__global__ void __launch_bounds__(128, 1) vgemm_seg_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+                                                           const __nv_bfloat16 *__restrict__ A3,
+                                                           __nv_bfloat16 *V3, int64_t N, float scale, int32_t *st) {
+    constexpr int D = 256, KC = D / 64, NCH = 3 * KC, NS = VSegCfg::NS;
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar[NS];
+    __shared__ uint32_t tmem_base;
+    const int s = blockIdx.x;
+    if (s >= *S.nseg) return;
+    const int len = S.len[s];
+    const int64_t start = S.start[s];
+    const int nblk = len > 128 ? 2 : 1;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = tmem_base;
+    const __nv_bfloat16 *Xs = H + start * D;
+    const __nv_bfloat16 *Aseg = A3 + (size_t)s * 3 * D * D;
+    auto load = [&](int c, uint32_t sa) {
+        const int p = c / KC, kc = c % KC;
+        for (int e = tid; e < 256 * 8; e += 128) {
+            const int r = e >> 3, ch = e & 7;
+            const bool in = r < len;
+            const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
+            tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + kc * 64 + ch * 8, in ? 16u : 0u);
+            tc::cp_async16(sa + VSegCfg::X_BYTES + tc::kmajor_off(r, ch * 8),
+                           Aseg + (size_t)p * D * D + (size_t)r * D + kc * 64 + ch * 8, 16u);
+        }
+    };
+    constexpr uint32_t idesc = tc::idesc_bf16(128, 256, false, false);
+    bool ok = true;
+    for (int c = 0; c < NS - 1; ++c) {
+        load(c, base + (uint32_t)c * VSegCfg::STAGE);
+        tc::cp_async_commit();
+    }
+    for (int c = 0; c < NCH; ++c) {
+        const int cn = c + NS - 1;
+        if (cn < NCH) {
+            if (cn >= NS) ok &= tc::mbar_wait(&mbar[cn % NS], (uint32_t)((cn / NS) - 1) & 1u, st);
+            load(cn, base + (uint32_t)(cn % NS) * VSegCfg::STAGE);
+        }
+        tc::cp_async_commit();
+        tc::cp_async_wait<NS - 1>();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t sa = base + (uint32_t)(c % NS) * VSegCfg::STAGE, sb = sa + VSegCfg::X_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = tc::sdesc(sb + kk * 32, 16, 1024);
+                for (int b = 0; b < nblk; ++b)
+                    tc::mma_bf16(tbase + (uint32_t)(b * 256), tc::sdesc(sa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
+                                 bd, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc::mma_commit(&mbar[c % NS]);
+        }
+        __syncthreads();
+    }
+    ok &= tc::mbar_wait(&mbar[(NCH - 1) % NS], (uint32_t)((NCH - 1) / NS) & 1u, st);
+    ok = __syncthreads_and(ok) != 0;
+    tc::fence_after_sync();
+    if (ok) {
+        tc::cp_async_wait<0>();
+        __syncthreads();
+        uint8_t *stg = smraw + (base - tc::smem_u32(smraw));
+        constexpr int RS = 144;
+        __nv_bfloat16 *vb = V3 + (size_t)start * D;
+#pragma unroll 1
+        for (int cb = 0; cb < D; cb += 64) {
+#pragma unroll 1
+            for (int b = 0; b < nblk; ++b) {
+                const int row = b * 128 + warp * 32 + lane;
+#pragma unroll 1
+                for (int j = 0; j < 4; ++j) {
+                    float v[16];
+                    tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * 256 + cb + 16 * j), v);
+                    __align__(16) __nv_bfloat16 h[16], m[16], l[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) split3(scale * v[i], h[i], m[i], l[i]);
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(p == 0 ? h : (p == 1 ? m : l));
+                        uint4 *d = reinterpret_cast<uint4 *>(stg + (size_t)(p * 256 + row) * RS + j * 32);
+                        d[0] = src[0];
+                        d[1] = src[1];
+                    }
+                }
+            }
+            __syncthreads();
+            for (int e = tid; e < 3 * 256 * 8; e += 128) {
+                const int pr = e >> 3, ch = e & 7, p = pr >> 8, r = pr & 255;
+                if (r < len)
+                    *reinterpret_cast<uint4 *>(vb + (size_t)p * N * D + (size_t)r * D + cb + ch * 8) =
+                        *reinterpret_cast<const uint4 *>(stg + (size_t)pr * RS + ch * 16);
+            }
+            __syncthreads();
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 512);
+}
+
 struct KCfg {
     static constexpr int NS = 4;
     static constexpr uint32_t STAGE = 128 * 128 + 128 * 128;
@@ -481,8 +604,8 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(H, L.segs, L.P, L.Bscr, L.A3, nullptr, N,
                                                                          dR, st);
-    cudaFuncSetAttribute(vgemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VCfg<D>::SMEM);
-    vgemm_kernel<D><<<dim3((unsigned)ns, 2), 128, VCfg<D>::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, (float)c, st);
+    cudaFuncSetAttribute(vgemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VSegCfg::SMEM);
+    vgemm_seg_kernel<<<(unsigned)ns, 128, VSegCfg::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, (float)c, st);
     tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(H, L.segs, nullptr, nullptr, nullptr,
                                                                           L.V3, N, dR, st);
     count_launches(6);
