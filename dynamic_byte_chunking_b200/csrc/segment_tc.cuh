@@ -308,22 +308,24 @@ __global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__re
     if (warp == 0) tc::tmem_dealloc(tbase, D);
 }
 
-// V = c X_s A_s for a whole segment of up to 256 positions in one CTA (d = 256):
-// both 128-row blocks accumulate in TMEM (columns 0 and 256), so each piece of
-// A_s is read once per segment; written as three bf16 pieces through shared
-// memory in whole 128-byte row segments.
-struct VSegCfg {
+// Y = sqrt(c) X_s B_s for a whole segment of up to 256 positions in one CTA
+// (d = 256): both 128-row blocks accumulate in TMEM (columns 0 and 256), so
+// each piece of B_s is read once per segment.  B_s = L_s^{-T} is upper
+// triangular and was stored per 16-column panel for the rows above the
+// panel's end only; the loads zero-fill the rest.  Y is written as three bf16
+// pieces through shared memory in whole 128-byte row segments.
+struct YSegCfg {
     static constexpr int NS = 3;
-    static constexpr uint32_t X_BYTES = 2 * 128 * 128;         // 256 positions x 64 K
-    static constexpr uint32_t STAGE = X_BYTES + 256 * 128;     // + 256 rows of A x 64 K
+    static constexpr uint32_t X_BYTES = 2 * 128 * 128;         // 256 positions x 64 K (K-major)
+    static constexpr uint32_t STAGE = X_BYTES + 4 * 8192;      // + 64 K x 256 columns of B (MN-major)
     static constexpr size_t SMEM = NS * STAGE + 1024;
 };
-static_assert(VSegCfg::NS * VSegCfg::STAGE >= 3u * 256u * 144u, "epilogue staging must fit in the stages");
+static_assert(YSegCfg::NS * YSegCfg::STAGE >= 3u * 256u * 144u, "epilogue staging must fit in the stages");
 
-__global__ void __launch_bounds__(128, 1) vgemm_seg_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
-                                                           const __nv_bfloat16 *__restrict__ A3,
-                                                           __nv_bfloat16 *V3, int64_t N, float scale, int32_t *st) {
-    constexpr int D = 256, KC = D / 64, NCH = 3 * KC, NS = VSegCfg::NS;
+__global__ void __launch_bounds__(128, 1) ygemm_seg_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+                                                           const __nv_bfloat16 *__restrict__ Bscr,
+                                                           __nv_bfloat16 *Y3, int64_t N, float scale, int32_t *st) {
+    constexpr int D = 256, KC = D / 64, NCH = 3 * KC, NS = YSegCfg::NS;
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[NS];
     __shared__ uint32_t tmem_base;
@@ -344,29 +346,35 @@ __global__ void __launch_bounds__(128, 1) vgemm_seg_kernel(const __nv_bfloat16 *
     tc::fence_after_sync();
     const uint32_t tbase = tmem_base;
     const __nv_bfloat16 *Xs = H + start * D;
-    const __nv_bfloat16 *Aseg = A3 + (size_t)s * 3 * D * D;
+    const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
     auto load = [&](int c, uint32_t sa) {
         const int p = c / KC, kc = c % KC;
-        for (int e = tid; e < 256 * 8; e += 128) {
+        for (int e = tid; e < 256 * 8; e += 128) {            // X: 256 positions x 8 units of 8 K
             const int r = e >> 3, ch = e & 7;
             const bool in = r < len;
             const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
             tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + kc * 64 + ch * 8, in ? 16u : 0u);
-            tc::cp_async16(sa + VSegCfg::X_BYTES + tc::kmajor_off(r, ch * 8),
-                           Aseg + (size_t)p * D * D + (size_t)r * D + kc * 64 + ch * 8, 16u);
+        }
+        const uint32_t sb = sa + YSegCfg::X_BYTES;
+        for (int e = tid; e < 64 * 32; e += 128) {            // B: 64 K rows x 32 units of 8 columns
+            const int k = e >> 5, n8 = e & 31;
+            const int kr = kc * 64 + k;
+            const bool nz = kr < (n8 >> 1) * 16 + 16;         // stored rows of the columns' panel
+            tc::cp_async16(sb + tc::mnmajor_off(n8 * 8, k, 8192),
+                           Bseg + (size_t)p * D * D + (size_t)(nz ? kr : 0) * D + n8 * 8, nz ? 16u : 0u);
         }
     };
-    constexpr uint32_t idesc = tc::idesc_bf16(128, 256, false, false);
+    constexpr uint32_t idesc = tc::idesc_bf16(128, 256, false, true);
     bool ok = true;
     for (int c = 0; c < NS - 1; ++c) {
-        load(c, base + (uint32_t)c * VSegCfg::STAGE);
+        load(c, base + (uint32_t)c * YSegCfg::STAGE);
         tc::cp_async_commit();
     }
     for (int c = 0; c < NCH; ++c) {
         const int cn = c + NS - 1;
         if (cn < NCH) {
             if (cn >= NS) ok &= tc::mbar_wait(&mbar[cn % NS], (uint32_t)((cn / NS) - 1) & 1u, st);
-            load(cn, base + (uint32_t)(cn % NS) * VSegCfg::STAGE);
+            load(cn, base + (uint32_t)(cn % NS) * YSegCfg::STAGE);
         }
         tc::cp_async_commit();
         tc::cp_async_wait<NS - 1>();
@@ -374,10 +382,10 @@ __global__ void __launch_bounds__(128, 1) vgemm_seg_kernel(const __nv_bfloat16 *
         __syncthreads();
         if (tid == 0) {
             tc::fence_after_sync();
-            const uint32_t sa = base + (uint32_t)(c % NS) * VSegCfg::STAGE, sb = sa + VSegCfg::X_BYTES;
+            const uint32_t sa = base + (uint32_t)(c % NS) * YSegCfg::STAGE, sb = sa + YSegCfg::X_BYTES;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bd = tc::sdesc(sb + kk * 32, 16, 1024);
+                const uint64_t bd = tc::sdesc(sb + kk * 2048, 8192, 1024);
                 for (int b = 0; b < nblk; ++b)
                     tc::mma_bf16(tbase + (uint32_t)(b * 256), tc::sdesc(sa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
                                  bd, idesc, (c > 0 || kk > 0) ? 1u : 0u);
@@ -394,7 +402,7 @@ __global__ void __launch_bounds__(128, 1) vgemm_seg_kernel(const __nv_bfloat16 *
         __syncthreads();
         uint8_t *stg = smraw + (base - tc::smem_u32(smraw));
         constexpr int RS = 144;
-        __nv_bfloat16 *vb = V3 + (size_t)start * D;
+        __nv_bfloat16 *yb = Y3 + (size_t)start * D;
 #pragma unroll 1
         for (int cb = 0; cb < D; cb += 64) {
 #pragma unroll 1
@@ -420,7 +428,7 @@ __global__ void __launch_bounds__(128, 1) vgemm_seg_kernel(const __nv_bfloat16 *
             for (int e = tid; e < 3 * 256 * 8; e += 128) {
                 const int pr = e >> 3, ch = e & 7, p = pr >> 8, r = pr & 255;
                 if (r < len)
-                    *reinterpret_cast<uint4 *>(vb + (size_t)p * N * D + (size_t)r * D + cb + ch * 8) =
+                    *reinterpret_cast<uint4 *>(yb + (size_t)p * N * D + (size_t)r * D + cb + ch * 8) =
                         *reinterpret_cast<const uint4 *>(stg + (size_t)pr * RS + ch * 16);
             }
             __syncthreads();
@@ -557,9 +565,8 @@ constexpr int kLmaxTmem = 256;
 struct Layout3 {
     Segs segs;
     float *P;               // per segment: [D][D] Gram -> c-scaled prefix
-    __nv_bfloat16 *Bscr;    // per segment: [3][D][D] pieces of L^{-T}
-    __nv_bfloat16 *A3;      // per segment: [3][D][D] pieces of M_s^{-1}
-    __nv_bfloat16 *V3;      // [3][N][D] pieces of c X_s M_s^{-1}
+    __nv_bfloat16 *Bscr;    // per segment: [3][D][D] pieces of B = L^{-T} (rows below a panel unstored)
+    __nv_bfloat16 *Y3;      // [3][N][D] pieces of Y = sqrt(c) X_s B_s
     size_t bytes;
 };
 
@@ -575,8 +582,7 @@ inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d) {
     L.segs.nseg = c.take<int32_t>(1);
     L.P = c.take<float>((size_t)ns * d * d);
     L.Bscr = c.take<__nv_bfloat16>((size_t)ns * 3 * d * d);
-    L.A3 = c.take<__nv_bfloat16>((size_t)ns * 3 * d * d);
-    L.V3 = c.take<__nv_bfloat16>((size_t)3 * N * d + 8);
+    L.Y3 = c.take<__nv_bfloat16>((size_t)3 * N * d + 8);
     L.bytes = c.off;
     return L;
 }
@@ -602,12 +608,11 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(H, L.segs, L.P, L.Bscr, L.A3, nullptr, N,
-                                                                         dR, st);
-    cudaFuncSetAttribute(vgemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)VSegCfg::SMEM);
-    vgemm_seg_kernel<<<(unsigned)ns, 128, VSegCfg::SMEM, stream>>>(H, L.segs, L.A3, L.V3, N, (float)c, st);
-    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(H, L.segs, nullptr, nullptr, nullptr,
-                                                                          L.V3, N, dR, st);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, dR, st);
+    cudaFuncSetAttribute(ygemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)YSegCfg::SMEM);
+    ygemm_seg_kernel<<<(unsigned)ns, 128, YSegCfg::SMEM, stream>>>(H, L.segs, L.Bscr, L.Y3, N, (float)std::sqrt(c),
+                                                                   st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, nullptr, L.Y3, N, dR, st);
     count_launches(6);
     return launch_status();
 }

@@ -16,14 +16,15 @@
 // accurate to fp32 (hi.hi, hi.mid, mid.hi, hi.lo, lo.hi, mid.mid), K = 16.
 // Two uses:
 //
-//  * FACTOR (segment start state M_s = I + P_s): the upper triangle, which
-//    starts at zero, carries B = L^{-T} along (row i of the identity solved
-//    against the factor, B_ii = 1 / L_ii), so one sweep yields both; the
-//    panels of B are saved and A = B B^T = M_s^{-1} is formed at the end on
-//    tcgen05 and stored as three bf16 pieces.
-//  * INSEG (one segment): G' = X (c V)^T is accumulated straight into TMEM
-//    (V = X_s A_s in pieces), factored in place, and the excess of each
-//    column gives dR_t = log1p(e_t) / 2.
+//  * FACTOR (segment start state M_s = I + P_s = L L^T): the upper triangle,
+//    which starts at zero, carries B = L^{-T} along (row i of the identity
+//    solved against the factor, B_ii = 1 / L_ii), so one sweep yields it;
+//    the panels of B are stored as three bf16 pieces.  Since
+//    M_s^{-1} = B B^T, the whitened rows Y = sqrt(c) X_s B give the segment's
+//    problem c X_s M_s^{-1} X_s^T = Y Y^T.
+//  * INSEG (one segment): G' = Y Y^T (Y in three pieces, six piece
+//    products) is accumulated straight into TMEM, I + G' is factored in
+//    place, and the excess of each column gives dR_t = log1p(e_t) / 2.
 #pragma once
 
 #include "tc.cuh"
@@ -33,10 +34,9 @@ namespace cr {
 
 struct TmemChol {
     static constexpr int NT = 256;
-    static constexpr uint32_t XT = 128 * 128;             // 128-row x 64-K bf16 tile
     static constexpr uint32_t PIECE = 256 * 128;          // 256-row x 64-K bf16 tile
     static constexpr uint32_t PANEL = 3 * PIECE;          // staged panel (three pieces)
-    static constexpr uint32_t GSTAGE = 2 * XT + PIECE;    // G' GEMM stage: X (two row blocks) + V piece
+    static constexpr uint32_t GSTAGE = 3 * PIECE;         // G' GEMM stage: the three pieces of Y, 64 K
     static constexpr uint32_t REGION = (2 * GSTAGE > PANEL) ? 2 * GSTAGE : PANEL;
     static constexpr size_t SMEM = REGION + 1024;
 };
@@ -151,8 +151,8 @@ __device__ __forceinline__ uint32_t idesc_neg(int N) { return tc::idesc_bf16(128
 
 template <bool FACTOR>
 __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
-    const __nv_bfloat16 *__restrict__ H, Segs S, const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr,
-    __nv_bfloat16 *A3, const __nv_bfloat16 *__restrict__ V3, int64_t N, float *dR, int32_t *st) {
+    Segs S, const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr, const __nv_bfloat16 *__restrict__ Y3,
+    int64_t N, float *dR, int32_t *st) {
     constexpr int D = 256;
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[2];
@@ -209,22 +209,19 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             }
             tc::tmem_wait_st();
         } else {
-            // G' = X (c V)^T over 3 pieces x (D/64) feature chunks, two stages
-            const __nv_bfloat16 *X = H + start * D;
-            constexpr int KC = D / 64, NCH = 3 * KC;
+            // G' = Y Y^T: per 64-feature chunk the three pieces of the segment's Y rows, six piece
+            // products; rows 0..127 only need columns 0..127 (the lower triangle); two stages
+            constexpr int NCH = D / 64;
             auto load = [&](int c, uint32_t sb) {
-                const int p = c / KC, kc = c % KC;
-                for (int e = tid; e < 256 * 8; e += TmemChol::NT) {
-                    const int r = e >> 3, ch = e & 7;
+                for (int e = tid; e < 3 * 256 * 8; e += TmemChol::NT) {
+                    const int p = e >> 11, r = (e >> 3) & 255, ch = e & 7;
                     const bool in = r < len;
-                    const __nv_bfloat16 *gx = X + (size_t)(in ? r : 0) * D + kc * 64 + ch * 8;
-                    const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : TmemChol::XT + tc::kmajor_off(r - 128, ch * 8);
-                    tc::cp_async16(sb + xo, gx, in ? 16u : 0u);
-                    const __nv_bfloat16 *gv = V3 + (size_t)p * N * D + (size_t)(start + (in ? r : 0)) * D + kc * 64 + ch * 8;
-                    tc::cp_async16(sb + 2 * TmemChol::XT + tc::kmajor_off(r, ch * 8), gv, in ? 16u : 0u);
+                    const __nv_bfloat16 *gy = Y3 + (size_t)p * N * D + (size_t)(start + (in ? r : 0)) * D + c * 64 + ch * 8;
+                    tc::cp_async16(sb + (uint32_t)p * TmemChol::PIECE + tc::kmajor_off(r, ch * 8), gy, in ? 16u : 0u);
                 }
             };
-            constexpr uint32_t idg = tc::idesc_bf16(128, 256, false, false);
+            constexpr uint32_t idg0 = tc::idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idg1 = tc::idesc_bf16(128, 256, false, false);
             load(0, region);
             tc::cp_async_commit();
             for (int c = 0; c < NCH; ++c) {
@@ -243,12 +240,18 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     tc::fence_after_sync();
                     const uint32_t sb = region + (uint32_t)(c & 1) * TmemChol::GSTAGE;
 #pragma unroll
-                    for (int b = 0; b < 2; ++b)
+                    for (int pr = 0; pr < 6; ++pr) {
+                        const uint32_t pa = sb + (uint32_t)pair_a(pr) * TmemChol::PIECE;
+                        const uint32_t pb = sb + (uint32_t)pair_b(pr) * TmemChol::PIECE;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc::mma_bf16(tbase + (uint32_t)(b * 256), tc::sdesc(sb + b * TmemChol::XT + kk * 32, 16, 1024),
-                                         tc::sdesc(sb + 2 * TmemChol::XT + kk * 32, 16, 1024), idg,
-                                         (c > 0 || kk > 0) ? 1u : 0u);
+                        for (int b = 0; b < 2; ++b)
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc::mma_bf16(tbase + (uint32_t)(b * 256),
+                                             tc::sdesc(pa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
+                                             tc::sdesc(pb + kk * 32, 16, 1024), b == 0 ? idg0 : idg1,
+                                             (c > 0 || pr > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc::mma_commit(&mbar[c & 1]);
                 }
                 __syncthreads();
@@ -417,78 +420,6 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
         }
         if (!ok) break;
 
-        // ---------------- FACTOR: A = B B^T from the saved panels, split into pieces
-        if (FACTOR) {
-            for (int q = 0; q < D / 64; ++q) {
-                for (int e = tid; e < 3 * 256 * 8; e += TmemChol::NT) {
-                    const int p = e / 2048, r = (e >> 3) & 255, ch = e & 7;
-                    const bool nz = r < q * 64 + (ch >> 1) * 16 + 16;   // rows below a panel are zero there
-                    const __nv_bfloat16 *gsrc = Bs + (size_t)p * D * D + (size_t)(nz ? r : 0) * D + q * 64 + ch * 8;
-                    tc::cp_async16(region + (uint32_t)p * TmemChol::PIECE + tc::kmajor_off(r, ch * 8), gsrc,
-                                   nz ? 16u : 0u);
-                }
-                tc::cp_async_commit();
-                tc::cp_async_wait<0>();
-                tc::fence_async_smem();
-                __syncthreads();
-                if (tid == 0) {
-                    tc::fence_after_sync();
-                    constexpr uint32_t idp = tc::idesc_bf16(128, 256, false, false);
-                    for (int b = 0; b < 2; ++b) {
-                        if (b == 1 && q < 2) continue;          // rows 128.. of B vanish in columns < 128
-                        issue_split_mma(tbase + (uint32_t)(b * 256), region, region, b * 128, 0, idp,
-                                        b == 0 ? (q == 0) : (q == 2));
-                    }
-                    tc::mma_commit(&mbar[0]);
-                }
-                ok &= tc::mbar_wait(&mbar[0], ph0, st);
-                ph0 ^= 1;
-                tc::fence_after_sync();
-                ok = __syncthreads_and(ok) != 0;
-                if (!ok) break;
-            }
-            if (!ok) break;
-            // A -> three bf16 pieces, staged per 64-column block in shared memory (row-major, 144-byte
-            // rows) and written out as whole 128-byte row segments
-            __nv_bfloat16 *Ag = A3 + (size_t)s * 3 * D * D;
-            uint8_t *stg = smraw + (region - tc::smem_u32(smraw));
-            constexpr int RS = 144;
-#pragma unroll 1
-            for (int cb = 0; cb < D; cb += 64) {
-#pragma unroll 1
-                for (int j = 0; j < 4; ++j) {
-                    float t16[16];
-                    tc::tmem_ld16(trow + (uint32_t)(cb + 16 * j), t16);
-                    uint32_t hh[8], mm[8], ll[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint16_t h0, m0, l0, h1, m1, l1;
-                        split3v(t16[2 * q], h0, m0, l0);
-                        split3v(t16[2 * q + 1], h1, m1, l1);
-                        hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                        mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
-                        ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-                    }
-                    uint4 *d0 = reinterpret_cast<uint4 *>(stg + (size_t)row * RS + j * 32);
-                    uint4 *d1 = reinterpret_cast<uint4 *>(stg + (size_t)(256 + row) * RS + j * 32);
-                    uint4 *d2 = reinterpret_cast<uint4 *>(stg + (size_t)(512 + row) * RS + j * 32);
-                    d0[0] = make_uint4(hh[0], hh[1], hh[2], hh[3]); d0[1] = make_uint4(hh[4], hh[5], hh[6], hh[7]);
-                    d1[0] = make_uint4(mm[0], mm[1], mm[2], mm[3]); d1[1] = make_uint4(mm[4], mm[5], mm[6], mm[7]);
-                    d2[0] = make_uint4(ll[0], ll[1], ll[2], ll[3]); d2[1] = make_uint4(ll[4], ll[5], ll[6], ll[7]);
-                }
-                __syncthreads();
-                for (int e = tid; e < 3 * 256 * 8; e += TmemChol::NT) {
-                    const int pr = e >> 3, ch = e & 7;                 // piece-row (piece * 256 + row), chunk
-                    const uint4 x = *reinterpret_cast<const uint4 *>(stg + (size_t)pr * RS + ch * 16);
-                    const int pc = pr >> 8, r = pr & 255;
-                    *reinterpret_cast<uint4 *>(Ag + (size_t)pc * D * D + (size_t)r * D + cb + ch * 8) = x;
-                }
-                __syncthreads();
-            }
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
-        }
     }
     tc::fence_before_sync();
     __syncthreads();
