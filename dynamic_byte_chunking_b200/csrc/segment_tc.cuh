@@ -322,7 +322,7 @@ struct YSegCfg {
 };
 static_assert(YSegCfg::NS * YSegCfg::STAGE >= 3u * 256u * 144u, "epilogue staging must fit in the stages");
 
-__global__ void __launch_bounds__(128, 1) ygemm_seg_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+__global__ void __launch_bounds__(256, 1) ygemm_seg_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
                                                            const __nv_bfloat16 *__restrict__ Bscr,
                                                            __nv_bfloat16 *Y3, int64_t N, float scale, int32_t *st) {
     constexpr int D = 256, KC = D / 64, NCH = 3 * KC, NS = YSegCfg::NS;
@@ -349,14 +349,14 @@ __global__ void __launch_bounds__(128, 1) ygemm_seg_kernel(const __nv_bfloat16 *
     const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
     auto load = [&](int c, uint32_t sa) {
         const int p = c / KC, kc = c % KC;
-        for (int e = tid; e < 256 * 8; e += 128) {            // X: 256 positions x 8 units of 8 K
+        for (int e = tid; e < 256 * 8; e += 256) {            // X: 256 positions x 8 units of 8 K
             const int r = e >> 3, ch = e & 7;
             const bool in = r < len;
             const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
             tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + kc * 64 + ch * 8, in ? 16u : 0u);
         }
         const uint32_t sb = sa + YSegCfg::X_BYTES;
-        for (int e = tid; e < 64 * 32; e += 128) {            // B: 64 K rows x 32 units of 8 columns
+        for (int e = tid; e < 64 * 32; e += 256) {            // B: 64 K rows x 32 units of 8 columns
             const int k = e >> 5, n8 = e & 31;
             const int kr = kc * 64 + k;
             const bool nz = kr < (n8 >> 1) * 16 + 16;         // stored rows of the columns' panel
@@ -403,15 +403,16 @@ __global__ void __launch_bounds__(128, 1) ygemm_seg_kernel(const __nv_bfloat16 *
         uint8_t *stg = smraw + (base - tc::smem_u32(smraw));
         constexpr int RS = 144;
         __nv_bfloat16 *yb = Y3 + (size_t)start * D;
+        // warps 0-3 read the first row block's lanes, warps 4-7 the second's (TMEM columns + 256)
+        const int b = warp >> 2, lg = warp & 3;
+        const int row = b * 128 + lg * 32 + lane;
 #pragma unroll 1
         for (int cb = 0; cb < D; cb += 64) {
-#pragma unroll 1
-            for (int b = 0; b < nblk; ++b) {
-                const int row = b * 128 + warp * 32 + lane;
+            if (b < nblk) {                                       // warp-uniform
 #pragma unroll 1
                 for (int j = 0; j < 4; ++j) {
                     float v[16];
-                    tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * 256 + cb + 16 * j), v);
+                    tc::tmem_ld16(tbase + ((uint32_t)(lg * 32) << 16) + (uint32_t)(b * 256 + cb + 16 * j), v);
                     __align__(16) __nv_bfloat16 h[16], m[16], l[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) split3(scale * v[i], h[i], m[i], l[i]);
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(128, 1) ygemm_seg_kernel(const __nv_bfloat16 *
                 }
             }
             __syncthreads();
-            for (int e = tid; e < 3 * 256 * 8; e += 128) {
+            for (int e = tid; e < 3 * 256 * 8; e += 256) {
                 const int pr = e >> 3, ch = e & 7, p = pr >> 8, r = pr & 255;
                 if (r < len)
                     *reinterpret_cast<uint4 *>(yb + (size_t)p * N * D + (size_t)r * D + cb + ch * 8) =
@@ -610,7 +611,7 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, dR, st);
     cudaFuncSetAttribute(ygemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)YSegCfg::SMEM);
-    ygemm_seg_kernel<<<(unsigned)ns, 128, YSegCfg::SMEM, stream>>>(H, L.segs, L.Bscr, L.Y3, N, (float)std::sqrt(c),
+    ygemm_seg_kernel<<<(unsigned)ns, 256, YSegCfg::SMEM, stream>>>(H, L.segs, L.Bscr, L.Y3, N, (float)std::sqrt(c),
                                                                    st);
     tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, nullptr, L.Y3, N, dR, st);
     count_launches(6);

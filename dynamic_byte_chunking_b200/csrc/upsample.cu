@@ -115,7 +115,7 @@ struct BinTC {
 };
 
 template <class IN>
-__global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16 *__restrict__ G, int64_t dg,
+__global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16 *__restrict__ G, int64_t dg,
                                                              const IN *__restrict__ H, int64_t dl,
                                                              const __nv_bfloat16 *__restrict__ W, int nbins,
                                                              Layout L, float *__restrict__ S, int32_t *st) {
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
     const int64_t n0 = (int64_t)blockIdx.y * 256;
     const int nt = (int)(dl - n0 < 256 ? dl - n0 : 256);      // multiple of 64
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    {
+    if (tid < 128) {
         const int p = tid < cnt ? L.perm[r0 + tid] : -1;
         pos[tid] = p;
         grow[tid] = p >= 0 ? L.chunk[p] : -1;
@@ -152,13 +152,13 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
     const int nb8 = nt / 8;
     auto load = [&](int c, uint32_t sa) {
         const uint32_t sb = sa + BinTC::A_BYTES;
-        for (int e = tid; e < 128 * 8; e += 128) {
+        for (int e = tid; e < 128 * 8; e += 256) {
             const int r = e >> 3, ch = e & 7;
             const int g = grow[r];
             const __nv_bfloat16 *src = G + (size_t)(g >= 0 ? g : 0) * dg + c * 64 + ch * 8;
             tc::cp_async16(sa + tc::kmajor_off(r, ch * 8), src, g >= 0 ? 16u : 0u);
         }
-        for (int e = tid; e < 64 * nb8; e += 128) {
+        for (int e = tid; e < 64 * nb8; e += 256) {
             const int k = e / nb8, n8 = e - (e / nb8) * nb8;
             tc::cp_async16(sb + tc::mnmajor_off(n8 * 8, k, 8192), Wb + (size_t)(c * 64 + k) * dl + n8 * 8, 16u);
         }
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
         if (kPrefetchH && c == 0) {
             // residual rows of this tile: [128][nt] bf16, row-major (zeros for empty rows)
             const int nc = nt / 8;
-            for (int e = tid; e < 128 * nc; e += 128) {
+            for (int e = tid; e < 128 * nc; e += 256) {
                 const int r = e / nc, ch = e - (e / nc) * nc;
                 const int p = pos[r];
                 const IN *src = H + (size_t)(p >= 0 ? p : 0) * dl + n0 + ch * 8;
@@ -212,11 +212,13 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
         __syncthreads();
         float *tile = reinterpret_cast<float *>(smraw + (base - tc::smem_u32(smraw)));
         constexpr int LDT = 260;
-        const int r = warp * 32 + lane;
+        // warps w and w + 4 read the same 32 TMEM lanes, each half of the columns
+        const int lg = warp & 3, half = nt / 2;
+        const int r = lg * 32 + lane;
 #pragma unroll 1
-        for (int c0 = 0; c0 < nt; c0 += 16) {
+        for (int c0 = (warp >> 2) * half; c0 < (warp >> 2) * half + half; c0 += 16) {
             float v[16];
-            tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            tc::tmem_ld16(tbase + ((uint32_t)(lg * 32) << 16) + (uint32_t)c0, v);
             float4 *d = reinterpret_cast<float4 *>(tile + r * LDT + c0);
 #pragma unroll
             for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(128, 1) bin_gemm_tc_kernel(const __nv_bfloat16
         __syncthreads();
         const int nvec = nt / 8;                                   // 8 columns per lane
 #pragma unroll 1
-        for (int rr = warp; rr < 128; rr += 4) {
+        for (int rr = warp; rr < 128; rr += 8) {
             const int p = pos[rr];
             if (p < 0) continue;
             for (int c8 = lane; c8 < nvec; c8 += 32) {
@@ -271,13 +273,13 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
     if (dtype == DBC_BF16) {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)BinTC::smem<__nv_bfloat16>());
-        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 128, BinTC::smem<__nv_bfloat16>(), s>>>(
+        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 256, BinTC::smem<__nv_bfloat16>(), s>>>(
             static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
             static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
     } else {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)BinTC::smem<float>());
-        bin_gemm_tc_kernel<float><<<g, 128, BinTC::smem<float>(), s>>>(
+        bin_gemm_tc_kernel<float><<<g, 256, BinTC::smem<float>(), s>>>(
             static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
             static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
     }
