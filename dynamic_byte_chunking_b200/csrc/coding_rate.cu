@@ -227,7 +227,7 @@ struct GramTC {
 };
 
 template <int D>
-__global__ void __launch_bounds__(128, 1) gram_tc_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
+__global__ void __launch_bounds__(256, 1) gram_tc_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
                                                           float *aug, size_t mat_stride, int32_t *st) {
     using C = GramTC<D>;
     extern __shared__ uint8_t smraw[];
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(128, 1) gram_tc_kernel(const __nv_bfloat16 *__
     auto load = [&](int c) {
         const uint32_t sb = base + (uint32_t)(c % C::NS) * C::STAGE;
         const int t0 = c * C::KC;
-        for (int e = tid; e < C::KC * F8; e += 128) {
+        for (int e = tid; e < C::KC * F8; e += 256) {
             const int p = e / F8, f8 = e - (e / F8) * F8;
             const int pos = t0 + p;
             const __nv_bfloat16 *src = H + (start + (pos < len ? pos : 0)) * D + f8 * 8;
@@ -307,18 +307,24 @@ __global__ void __launch_bounds__(128, 1) gram_tc_kernel(const __nv_bfloat16 *__
     float *G = aug + (size_t)s * mat_stride;
     bool bad = false;
     if (ok) {
+        // 8 warps: warps w and w + 4 share the TMEM lanes of group w % 4 and take either one
+        // row block each (two blocks) or one half of the columns each (one block)
+        const int slot = warp >> 2, lg = warp & 3;
+        const int m = C::NMB == 2 ? slot : 0;
+        const int cbeg = C::NMB == 2 ? 0 : slot * (D / 2), cend = C::NMB == 2 ? D : cbeg + D / 2;
+        {
+            const int row = (mb0 + m) * 128 + lg * 32 + lane;
 #pragma unroll 1
-        for (int m = 0; m < C::NMB; ++m) {
-            const int row = (mb0 + m) * 128 + warp * 32 + lane;
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
+            for (int c0 = cbeg; c0 < cend; c0 += 16) {
                 float v[16];
-                tc::tmem_ld16(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)(m * D + c0), v);
+                tc::tmem_ld16(tbase + ((uint32_t)(lg * 32) << 16) + (uint32_t)(m * D + c0), v);
                 if (nchunks == 0) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) v[i] = 0.f;
                 }
-                if (row >= c0 && row < c0 + 16) bad |= !isfinite(v[row - c0]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (row == c0 + i) bad |= !isfinite(v[i]);
                 float4 *dst = reinterpret_cast<float4 *>(G + (size_t)row * D + c0);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -559,7 +565,7 @@ void launch_gram_tc(const __nv_bfloat16 *H, int64_t ns, const Segs &segs, float 
                     int32_t *st, cudaStream_t stream) {
     using C = GramTC<D>;
     cudaFuncSetAttribute(gram_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    gram_tc_kernel<D><<<dim3((unsigned)ns, (unsigned)C::GROUPS), 128, C::SMEM, stream>>>(H, segs, mats,
+    gram_tc_kernel<D><<<dim3((unsigned)ns, (unsigned)C::GROUPS), 256, C::SMEM, stream>>>(H, segs, mats,
                                                                                        mat_stride, st);
 }
 

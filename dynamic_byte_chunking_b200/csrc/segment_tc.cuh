@@ -506,7 +506,9 @@ __global__ void __launch_bounds__(128, 1) kgemm_kernel(const __nv_bfloat16 *__re
                         dst[q] = make_float4(c_rate * v[4 * q], c_rate * v[4 * q + 1], c_rate * v[4 * q + 2],
                                              c_rate * v[4 * q + 3]);
                 } else {
-                    for (int q = 0; q < 16 && j0 + q < len; ++q) G[c0 + q] = c_rate * v[q];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (j0 + q < len) G[c0 + q] = c_rate * v[q];
                 }
             }
         }
