@@ -23,6 +23,12 @@ Three independent evaluations:
   factor of M_t = I + c sum_{i<=t} h_i h_i^T, with the matrix determinant
   lemma det(M + c h h^T) = det(M)(1 + c h^T M^-1 h).
 
+Streaming continuation (:func:`dR_continue`): a stream delivered in blocks
+keeps, between blocks, the Gram sum S = sum of h h^T over everything seen so
+far; the next block's dR follow from the same definition with that prefix
+(R of the whole stream so far), so block-wise streaming reproduces the
+whole-sequence values exactly.
+
 This file is test infrastructure.  Only the test-suite, the smoke check and
 the benchmark's CPU-baseline leg may import it.
 """
@@ -30,7 +36,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["coding_rate", "coding_rate_T", "dR_prefix_logdet", "dR_chol_diag"]
+__all__ = ["coding_rate", "coding_rate_T", "dR_prefix_logdet", "dR_chol_diag", "dR_continue"]
 
 
 def _logdet_spd(A: np.ndarray) -> float:
@@ -92,3 +98,31 @@ def dR_chol_diag(H: np.ndarray, eps2: float) -> np.ndarray:
     G[np.diag_indices(T)] += 1.0
     L = np.linalg.cholesky(G)
     return np.log(np.diag(L))
+
+
+def dR_continue(S0: np.ndarray, H: np.ndarray, eps2: float, ts=None):
+    """dR of a new block H given the earlier positions' Gram sum S0 (float64).
+
+    dR_t = R(earlier + h_{0..t}) - R(earlier + h_{0..t-1}) with
+    R = 1/2 logdet(I + c S) and S the Gram sum of the positions included.
+    Returns (dR at ``ts`` (default all rows of H), S0 + H^T H).
+    """
+    H = np.asarray(H, dtype=np.float64)
+    T, d = H.shape
+    c = d / eps2
+    S0 = np.asarray(S0, dtype=np.float64)
+    ts = np.arange(T) if ts is None else np.asarray(ts, dtype=np.int64)
+    order = np.argsort(ts, kind="stable")
+    out = np.empty(len(ts), dtype=np.float64)
+    S = S0.copy()
+    upto = 0
+    I = np.eye(d)
+    for j in order:
+        t = int(ts[j])
+        if upto < t:
+            X = H[upto:t]
+            S += X.T @ X
+            upto = t
+        h = H[t]
+        out[j] = 0.5 * _logdet_spd(I + c * (S + np.outer(h, h))) - 0.5 * _logdet_spd(I + c * S)
+    return out, S0 + H.T @ H

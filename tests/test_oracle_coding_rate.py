@@ -237,3 +237,42 @@ def test_pins_catch_mutants(mut):
         except np.linalg.LinAlgError:
             bad = True
     assert bad
+
+
+# ---------------------------------------------------------------- streaming continuation
+def test_continuation_matches_whole_sequence_by_other_oracles():
+    """Blocks with a carried Gram sum give the whole sequence's dR (checked against the
+    Cholesky diagonal of the T x T Gram and the rank-1 recursion, both independent of it)."""
+    from oracle.coding_rate import dR_chol_diag, dR_continue
+    from oracle.rank1 import dR_rank1
+    rng = np.random.default_rng(7)
+    d, eps2 = 16, 0.5
+    H = (rng.standard_normal((150, d)) / np.sqrt(d)).astype(np.float32).astype(np.float64)   # the C oracle reads fp32
+    want = dR_chol_diag(H, eps2)
+    want3 = dR_rank1(H, np.array([0, 150]), eps2)
+    S = np.zeros((d, d))
+    got = []
+    for a, b in [(0, 1), (1, 40), (40, 41), (41, 150)]:      # blocks of 1, 39, 1, 109 positions
+        dr, S = dR_continue(S, H[a:b], eps2)
+        got.append(dr)
+    got = np.concatenate(got)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-13)
+    assert np.allclose(got, want3, rtol=1e-9, atol=1e-13)
+    assert np.allclose(S, H.T @ H, rtol=1e-13, atol=1e-13)
+
+
+def test_continuation_sampled_positions_and_empty_prefix():
+    from oracle.coding_rate import dR_continue, dR_prefix_logdet
+    rng = np.random.default_rng(8)
+    d, eps2 = 8, 0.25
+    H = rng.standard_normal((60, d)) / np.sqrt(d)
+    full, _ = dR_continue(np.zeros((d, d)), H, eps2)
+    # a zero prefix is the plain definition
+    assert np.allclose(full, dR_prefix_logdet(H, eps2), rtol=1e-12, atol=1e-14)
+    S20 = H[:20].T @ H[:20]
+    part, _ = dR_continue(S20, H[20:], eps2, ts=[0, 13, 39])
+    assert np.allclose(part, full[[20, 33, 59]], rtol=1e-12, atol=1e-14)
+    # a later byte never gains information: dR of a repeat is smaller than on a fresh state
+    again, _ = dR_continue(H.T @ H, H[:1], eps2)
+    fresh, _ = dR_continue(np.zeros((d, d)), H[:1], eps2)
+    assert again[0] < fresh[0]
