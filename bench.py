@@ -293,6 +293,25 @@ def run_rows(args):
         fl = 4.0 * d * d * N
         emit("A1 coding rate", fam, ms, positions_per_s=N / (ms * 1e-3), tflops=fl / (ms * 1e-3) / 1e12,
              frac_bf16_peak=fl / (ms * 1e-3) / 1e12 / tf)
+        if w.dense and d == 256 and w.dtype == "bf16":
+            # streaming continuation: the same rows fed as blocks of 256 positions with a carried state
+            blk = 256
+            Hs = H.view(rows, T, d)
+            blocks = [Hs[:, t0:t0 + blk, :].contiguous() for t0 in range(0, T, blk)]
+            state = torch.zeros(rows, d, d, dtype=torch.float64, device=dev)
+            dRs = torch.empty(rows * blk, dtype=torch.float32, device=dev)
+            wss = torch.empty(max(dbc.chunk_coding_rate_stream_workspace(rows, blk, t0, d)
+                                  for t0 in range(0, T, blk)), dtype=torch.uint8, device=dev)
+
+            def stream_pass():
+                state.zero_()
+                for j, b in enumerate(blocks):
+                    dbc.chunk_coding_rate_stream(b, w.eps2, state, j * blk, dR=dRs, workspace=wss)
+
+            ms = _time(stream_pass, args.reps, flush, stream)
+            emit("NEXT-2 streaming coding rate (blocks of 256)", fam, ms, positions_per_s=N / (ms * 1e-3),
+                 blocks=len(blocks), us_per_block=ms * 1e3 / len(blocks), tflops=fl / (ms * 1e-3) / 1e12)
+            del blocks, state, dRs, wss
         Kt = torch.from_numpy(w.K).to(dev)
         total = int(np.minimum(w.K, w.lengths).sum())
         idx = torch.empty(total, dtype=torch.int64, device=dev)

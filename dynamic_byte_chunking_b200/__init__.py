@@ -23,7 +23,8 @@ from typing import Optional
 
 __all__ = [
     "DbcError", "lib", "lib_path", "version", "status_string", "launch_count",
-    "chunk_coding_rate", "chunk_coding_rate_workspace", "chunk_topk_select",
+    "chunk_coding_rate", "chunk_coding_rate_workspace", "chunk_coding_rate_stream",
+    "chunk_coding_rate_stream_workspace", "chunk_topk_select",
     "chunk_gather", "chunk_upsample", "chunk_upsample_workspace", "chunk_upsample_noalloc",
     "chunk_upsample_backward", "chunk_upsample_backward_workspace", "chunk_gather_backward",
     "hnet_route", "hnet_route_workspace", "chunk",
@@ -47,6 +48,8 @@ _SIGS = {
     "dbc_launch_count": (ctypes.c_uint64, []),
     "chunk_coding_rate_workspace": (_sz, [_i64, _i64, _i64, _i64]),
     "chunk_coding_rate": (_int, [_vp, _int, _vp, _i64, _i64, _i64, _i64, _f32, _vp, _vp, _sz, _vp, _vp]),
+    "chunk_coding_rate_stream_workspace": (_sz, [_i64, _i64, _i64, _i64]),
+    "chunk_coding_rate_stream": (_int, [_vp, _int, _i64, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "chunk_topk_select_workspace": (_sz, [_i64]),
     "chunk_topk_select": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "chunk_gather": (_int, [_vp, _int, _vp, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp,
@@ -180,6 +183,32 @@ def chunk_coding_rate(H, eps2: float, *, offsets=None, T: Optional[int] = None, 
     rc = lib().chunk_coding_rate(_ptr(H2), _dtype_code(H2), _ptr(offsets), rows, T, N, d, float(eps2),
                                  _ptr(dR), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
     _check("chunk_coding_rate", rc)
+    return dR
+
+
+def chunk_coding_rate_stream_workspace(streams: int, n: int, t0: int, d: int) -> int:
+    return int(lib().chunk_coding_rate_stream_workspace(streams, n, t0, d))
+
+
+def chunk_coding_rate_stream(H, eps2: float, state, t0: int, *, dR=None, workspace=None, dev_status=None,
+                             stream=None):
+    """dR (fp32 [streams * n]) of n new positions per stream ([streams, n, 256] bf16) that continue
+    streams which already consumed t0 positions; ``state`` (float64 [streams, 256, 256], the Gram sum
+    of everything seen, zero for new streams) is advanced in place."""
+    torch = _torch()
+    _require_cuda(H, state)
+    if H.dim() != 3:
+        raise ValueError("H must be [streams, n, d]")
+    streams, n, d = H.shape
+    if state.dtype != torch.float64 or tuple(state.shape) != (streams, d, d) or not state.is_contiguous():
+        raise TypeError("state must be a contiguous float64 [streams, d, d] tensor")
+    H2 = H.contiguous()
+    if dR is None:
+        dR = torch.empty(streams * n, dtype=torch.float32, device=H.device)
+    ws = _workspace(chunk_coding_rate_stream_workspace(streams, n, t0, d), H.device, workspace)
+    rc = lib().chunk_coding_rate_stream(_ptr(H2), _dtype_code(H2), streams, n, d, int(t0), float(eps2), _ptr(state),
+                                        _ptr(dR), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
+    _check("chunk_coding_rate_stream", rc)
     return dR
 
 

@@ -674,3 +674,31 @@ extern "C" dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t 
                        dev_status, s);
     return cr::run(static_cast<const float *>(H), offsets, rows, T, N, d, eps2, dR, L, dev_status, s);
 }
+
+// Streaming continuation: n new positions of each of `streams` streams that have
+// already consumed t0 positions (bf16, d = 256).
+extern "C" size_t chunk_coding_rate_stream_workspace(int64_t streams, int64_t n, int64_t t0, int64_t d) {
+    if (streams < 0 || n < 0 || t0 < 0 || d != 256) return 0;
+    int64_t k1 = 0, cnt = 0;
+    cr::stream_pieces(t0, n, k1, cnt);
+    return cr::carve3(nullptr, streams, streams * n, d, streams * cnt).bytes;
+}
+
+extern "C" dbc_status chunk_coding_rate_stream(const void *H, int dtype, int64_t streams, int64_t n, int64_t d,
+                                               int64_t t0, float eps2, double *state, float *dR, void *ws,
+                                               size_t ws_bytes, int32_t *dev_status, dbc_stream_t stream) {
+    if (streams < 0 || n < 0 || t0 < 0 || !(eps2 > 0.f) || !isfinite(eps2)) return DBC_ERR_INVALID_ARG;
+    if (dtype != DBC_BF16 || d != 256) return DBC_ERR_UNSUPPORTED;
+    if (streams == 0 || n == 0) return DBC_OK;
+    if (!H || !dR || !state || !aligned16(H) || !aligned16(state)) return DBC_ERR_INVALID_ARG;
+    if (streams * n > INT32_MAX || t0 > ((int64_t)1 << 40)) return DBC_ERR_UNSUPPORTED;
+    int64_t k1 = 0, cnt = 0;
+    cr::stream_pieces(t0, n, k1, cnt);
+    if (streams * cnt > INT32_MAX / 2) return DBC_ERR_UNSUPPORTED;
+    const cr::Layout3 need = cr::carve3(nullptr, streams, streams * n, d, streams * cnt);
+    if (!ws || ws_bytes < need.bytes || (reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)))
+        return DBC_ERR_WORKSPACE;
+    return cr::run_tmem_stream(static_cast<const __nv_bfloat16 *>(H), streams, n, t0, k1, cnt, eps2, state, dR,
+                               cr::carve3(ws, streams, streams * n, d, streams * cnt), dev_status,
+                               reinterpret_cast<cudaStream_t>(stream));
+}

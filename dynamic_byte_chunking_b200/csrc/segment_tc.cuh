@@ -573,9 +573,11 @@ struct Layout3 {
     size_t bytes;
 };
 
-inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d) {
+// ns_given >= 0: exactly that many segments (the streaming continuation), else
+// the batch upper bound.
+inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d, int64_t ns_given = -1) {
     Carver c(ws);
-    const int64_t ns = nseg_upper(rows, N, kLmaxTmem);
+    const int64_t ns = ns_given >= 0 ? ns_given : nseg_upper(rows, N, kLmaxTmem);
     Layout3 L;
     L.segs.start = c.take<int64_t>(ns);
     L.segs.len = c.take<int32_t>(ns);
@@ -608,6 +610,101 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
     prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
         L.segs, L.P, D, c, (size_t)D * D);
+    const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
+    cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
+    cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, dR, st);
+    cudaFuncSetAttribute(ygemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)YSegCfg::SMEM);
+    ygemm_seg_kernel<<<(unsigned)ns, 256, YSegCfg::SMEM, stream>>>(H, L.segs, L.Bscr, L.Y3, N, (float)std::sqrt(c),
+                                                                   st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, nullptr, L.Y3, N, dR, st);
+    count_launches(6);
+    return launch_status();
+}
+
+// ================================================================ streaming continuation (d = 256)
+// `streams` rows of n new positions each continue streams that have already
+// consumed t0 positions; their Gram sums S (float64, [streams][D][D], the
+// caller's buffer) are the start state and are advanced by the new block.  The
+// new positions are cut at the same absolute segment boundaries as a whole
+// sequence (0, 64, 128, then every multiple of 256), so a segment is never
+// longer than the prefix before it, and the values equal the whole sequence's.
+
+// First boundary above t0 (index k1) and the number of pieces of [t0, t0 + n).
+inline void stream_pieces(int64_t t0, int64_t n, int64_t &k1, int64_t &cnt) {
+    const int k0 = seg_k0(kLmaxTmem);
+    if (t0 < seg_bound(k0, kLmaxTmem)) {
+        k1 = 0;
+        while (seg_bound(k1, kLmaxTmem) <= t0) ++k1;
+    } else {
+        k1 = k0 + t0 / kLmaxTmem;           // seg_bound(k) = 256 (k - k0 + 1) > t0
+    }
+    cnt = n > 0 ? 1 : 0;
+    while (n > 0 && seg_bound(k1 + cnt - 1, kLmaxTmem) < t0 + n) ++cnt;
+}
+
+__global__ void __launch_bounds__(256) stream_seg_table_kernel(int64_t streams, int64_t n, int64_t t0, int64_t k1,
+                                                               int64_t cnt, Segs S) {
+    const int64_t total = streams * cnt;
+    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < total; s += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = s / cnt, j = s - r * cnt;
+        const int64_t a = j == 0 ? t0 : seg_bound(k1 + j - 1, kLmaxTmem);
+        const int64_t e = j + 1 < cnt ? seg_bound(k1 + j, kLmaxTmem) : t0 + n;
+        S.start[s] = r * n + (a - t0);
+        S.len[s] = (int32_t)(e - a);
+        S.row[s] = (int32_t)r;
+        S.k[s] = (int32_t)j;
+        if (j == 0) S.row_seg0[r] = (int32_t)s;
+        if (s == 0) {
+            S.row_seg0[streams] = (int32_t)total;
+            *S.nseg = (int32_t)total;
+        }
+    }
+}
+
+// P_s = c (S_row + sum of the row's earlier segment Grams), running sums in
+// float64 starting from the carried state, which is advanced to the end.
+__global__ void __launch_bounds__(256) prefix_stream_kernel(Segs S, float *P, double *state, int64_t d, double c) {
+    const int64_t r = blockIdx.x;
+    const int64_t e4 = (int64_t)blockIdx.y * 256 + threadIdx.x;        // float4 index
+    if (e4 * 4 >= d * d) return;
+    double *sr = state + (size_t)r * d * d + 4 * e4;
+    double acc[4] = {sr[0], sr[1], sr[2], sr[3]};
+    const int s0 = S.row_seg0[r], s1 = S.row_seg0[r + 1];
+    for (int sb = s0; sb < s1; sb += 16) {
+        const int cnt = min(16, s1 - sb);
+        float4 g[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (q < cnt) g[q] = *reinterpret_cast<const float4 *>(P + (size_t)(sb + q) * d * d + 4 * e4);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (q < cnt) {
+                *reinterpret_cast<float4 *>(P + (size_t)(sb + q) * d * d + 4 * e4) =
+                    make_float4((float)(c * acc[0]), (float)(c * acc[1]), (float)(c * acc[2]), (float)(c * acc[3]));
+                acc[0] += (double)g[q].x;
+                acc[1] += (double)g[q].y;
+                acc[2] += (double)g[q].z;
+                acc[3] += (double)g[q].w;
+            }
+        }
+    }
+    sr[0] = acc[0]; sr[1] = acc[1]; sr[2] = acc[2]; sr[3] = acc[3];
+}
+
+inline dbc_status run_tmem_stream(const __nv_bfloat16 *H, int64_t streams, int64_t n, int64_t t0, int64_t k1,
+                                  int64_t cnt, float eps2, double *state, float *dR, const Layout3 &L, int32_t *st,
+                                  cudaStream_t stream) {
+    constexpr int D = 256;
+    const double c = (double)D / (double)eps2;
+    const int64_t ns = streams * cnt;
+    const int64_t N = streams * n;
+    const int sms = num_sms();
+    const int tgrid = (int)std::max<int64_t>(1, std::min<int64_t>((ns + 255) / 256, (int64_t)sms * 4));
+    stream_seg_table_kernel<<<tgrid, 256, 0, stream>>>(streams, n, t0, k1, cnt, L.segs);
+    launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
+    prefix_stream_kernel<<<dim3((unsigned)streams, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
+        L.segs, L.P, state, D, c);
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);

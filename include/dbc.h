@@ -104,6 +104,35 @@ DBC_API dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t *of
                              int32_t *dev_status, dbc_stream_t stream);
 
 /* -------------------------------------------------------------------------
+ * chunk_coding_rate_stream -- the marginal coding rate of streams delivered in
+ * blocks (causal use of the chunker).
+ *
+ * ByteFlow (summary "Prerequisites: lossy coding rate" and "Method steps",
+ * stage 2; notes "Key design 2"): dR_t = R(h_{0..t}) - R(h_{0..t-1}).  A
+ * stream that has already consumed t0 positions carries the Gram sum
+ * S = sum_{i < t0} h_i h_i^T of everything seen; the next n positions' dR are
+ * the whole sequence's values at t0 .. t0 + n - 1 (same definition, same
+ * segment boundaries 0, 64, 128, 256, 512, ... counted from the stream's start),
+ * and S is advanced by the block.  Selecting boundaries causally is left to
+ * the caller, e.g. chunk_topk_select over fixed windows of the stream.
+ *
+ * H        bf16 [streams, n, d] the new positions (d = 256 only).
+ * t0       positions each stream consumed before this call (all streams
+ *          equal); 0 starts the streams (state must then be zero).
+ * state    in/out float64 [streams, d, d]: S before the call, S after it.
+ *          Caller-owned, 16-byte aligned; zero it once per new stream.
+ * dR       out fp32 [streams, n].
+ * ws       workspace of chunk_coding_rate_stream_workspace(streams, n, t0, d)
+ *          bytes (it depends on t0 through the segment cut).
+ * Errors: INVALID_ARG, UNSUPPORTED (dtype other than bf16, d != 256),
+ * WORKSPACE, CUDA; device flags NONFINITE, TIMEOUT.
+ * ------------------------------------------------------------------------- */
+DBC_API size_t chunk_coding_rate_stream_workspace(int64_t streams, int64_t n, int64_t t0, int64_t d);
+DBC_API dbc_status chunk_coding_rate_stream(const void *H, int dtype, int64_t streams, int64_t n, int64_t d,
+                                            int64_t t0, float eps2, double *state, float *dR, void *ws,
+                                            size_t ws_bytes, int32_t *dev_status, dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
  * chunk_topk_select -- boundary positions per row.
  *
  * ByteFlow (notes "Key design 2"; summary stage 2): position 0 (BOS) is always

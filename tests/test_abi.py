@@ -94,3 +94,20 @@ def test_backward_argument_errors_return_before_launch(L):
     assert gb(None, 8, None, 8, None, None, 1, 0, None, 1, None, None) == 0
     import dynamic_byte_chunking_b200 as dbc
     assert dbc.chunk_upsample_backward_workspace(8, 65536, 16, 256) >= 2 * 65536 * 256 * 2
+
+
+def test_stream_argument_errors_and_workspace(L):
+    import dynamic_byte_chunking_b200 as dbc
+    f = L.chunk_coding_rate_stream
+    # fp32 input and d != 256 are not supported on this path
+    assert f(None, 0, 1, 8, 256, 0, ctypes.c_float(0.5), None, None, None, 0, None, None) == 2
+    assert f(None, 1, 1, 8, 128, 0, ctypes.c_float(0.5), None, None, None, 0, None, None) == 2
+    # negative t0, bad eps2
+    assert f(None, 1, 1, 8, 256, -1, ctypes.c_float(0.5), None, None, None, 0, None, None) == 1
+    assert f(None, 1, 1, 8, 256, 0, ctypes.c_float(0.0), None, None, None, 0, None, None) == 1
+    # an empty block is a no-op
+    assert f(None, 1, 1, 0, 256, 7, ctypes.c_float(0.5), None, None, None, 0, None, None) == 0
+    # the cut depends on t0: a block across 64 / 128 / 256 needs more segments than one inside [256, 512)
+    a = dbc.chunk_coding_rate_stream_workspace(4, 256, 1, 256)
+    b = dbc.chunk_coding_rate_stream_workspace(4, 256, 256, 256)
+    assert a > b > 0
