@@ -451,12 +451,19 @@ def main():
         if ev is not None:
             ev[4].record(stream)
 
+    def check_status(when):
+        # collective, so that every rank stops together when any rank saw a device flag
+        flags = st.to(torch.int64)
+        if pg:
+            pg.all_reduce(flags, op=pg.ReduceOp.MAX)
+        if flags.item() != 0:
+            raise RuntimeError(f"device status flags {flags.item():#x} {when}")
+
     for _ in range(args.warmup):
         flush.zero_()
         step(H)
     torch.cuda.synchronize()
-    if st.item() != 0:
-        raise RuntimeError(f"device status flags {st.item():#x} during warm-up")
+    check_status("during warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     gpu_id = str(local)
@@ -553,8 +560,7 @@ def main():
                "ms_per_step": ms_e2e}
 
     torch.cuda.synchronize()
-    if st.item() != 0:
-        raise RuntimeError(f"device status flags {st.item():#x}")
+    check_status("after the timed steps")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

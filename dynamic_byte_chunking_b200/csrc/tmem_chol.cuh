@@ -381,18 +381,31 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 // zero (in-segment mode, rows < j1)
                 stage_row16(region, row, a);
                 // factor mode: the diagonal rows' B entries right of the panel start from zero.
-                // tcgen05.ld/st are warp-collective (.sync.aligned), so the whole warp holding the
-                // block's half-warp reads its rows and writes them back, zeros for the block rows.
-                const int wrow0 = row - lane;                      // first row of this warp
-                if (FACTOR && wrow0 <= j0 && j0 < wrow0 + 32) {    // warp-uniform
+                // tcgen05.ld/st are warp-collective (.sync.aligned) and a warp may only address its
+                // lane group, so the two warps of the block rows' lane group (one per row block)
+                // read the columns past the panel and write them back, zeros for the block rows;
+                // each takes every other 32 columns, two loads in flight per wait.
+                const int gd = (j0 & 127) >> 5, bd = j0 >> 7;     // lane group, row block of the block
+                if (FACTOR && (warp & 3) == gd) {                 // warp-uniform
                     __syncwarp();
+                    const int lrow = bd * 128 + gd * 32 + lane;   // row of this lane in those columns
+                    const bool zero = lrow >= j0 && lrow < j0 + 16;
+                    const uint32_t tb = tbase + ((uint32_t)(gd * 32) << 16) + (uint32_t)(bd * 256);
 #pragma unroll 1
-                    for (int c0 = j1; c0 < D; c0 += 16) {
-                        float t[16];
-                        tc::tmem_ld16(trow + (uint32_t)c0, t);
+                    for (int c0 = j1 + 32 * (warp >> 2); c0 < D; c0 += 64) {
+                        const bool two = c0 + 16 < D;             // warp-uniform
+                        uint32_t r0[16], r1[16] = {};
+                        tc::tmem_ld16_nw(tb + (uint32_t)c0, r0);
+                        if (two) tc::tmem_ld16_nw(tb + (uint32_t)(c0 + 16), r1);
+                        tc::tmem_wait_ld();
+                        float t0[16], t1[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) t[i] = diag ? 0.f : t[i];
-                        tc::tmem_st16(trow + (uint32_t)c0, t);
+                        for (int i = 0; i < 16; ++i) {
+                            t0[i] = zero ? 0.f : __uint_as_float(r0[i]);
+                            t1[i] = zero ? 0.f : __uint_as_float(r1[i]);
+                        }
+                        tc::tmem_st16(tb + (uint32_t)c0, t0);
+                        if (two) tc::tmem_st16(tb + (uint32_t)(c0 + 16), t1);
                     }
                     tc::tmem_wait_st();
                 }
@@ -403,11 +416,12 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             if (j1 < n) {
                 if (tid == 0) {
                     tc::fence_after_sync();
-                    const uint32_t idn = idesc_neg(256 - j1);
 #pragma unroll
                     for (int b = 0; b < 2; ++b) {
                         if (!FACTOR && (b + 1) * 128 <= j1) continue;
-                        issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1), region, b * 128, j1, idn);
+                        // in-segment mode: the first row block only needs its lower triangle (columns < 128)
+                        const int nc = (!FACTOR && b == 0) ? 128 - j1 : 256 - j1;
+                        issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1), region, b * 128, j1, idesc_neg(nc));
                     }
                     tc::mma_commit(&mbar[0]);
                 }
