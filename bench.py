@@ -154,15 +154,33 @@ def cpu_baseline(w, min_seconds=10.0):
                       f"rank-1 C recursion for dR on all host threads, Top-K, gather, upsample; {dt:.2f} s"}
 
 
+def strip_comments(text):
+    """Kernel source without its comments: whole-line // comments, trailing // comments on lines
+    without string literals, and /* */ blocks; blank lines dropped, trailing blanks trimmed."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = []
+    for line in text.splitlines():
+        if line.lstrip().startswith("//"):
+            continue
+        if '"' not in line:
+            line = re.sub(r"\s*//.*$", "", line)
+        line = line.rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def csrc_sha256():
-    """Hash of the kernel sources, to tell whether a stored ncu capture still describes them."""
+    """Hash of the kernel sources with comments removed, to tell whether a stored ncu capture
+    still describes the kernels (a comment edit does not change what was measured)."""
     import glob
     import hashlib
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "dynamic_byte_chunking_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+        with open(f, encoding="utf-8") as fh:
             h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()
 
 

@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 for (int m = 0; m < 16; ++m) a[m] = 0.f;
             }
             if (FACTOR && row < j1) {
-                // B panel -> global pieces (rows >= j1 are zero here and never stored: the product
-                // B B^T below zero-fills them)
+                // B panel -> global pieces (rows >= j1 are zero here and never stored: the loads
+                // of the whitening GEMM zero-fill them)
                 __nv_bfloat16 *g = Bs + (size_t)row * D + j0;
 #pragma unroll
                 for (int k8 = 0; k8 < 2; ++k8) {

@@ -50,3 +50,13 @@ def test_source_hash_covers_every_kernel_file():
     assert len(h1) == 64 and h1 == bench.csrc_sha256()
     csrc = os.path.join(bench.ROOT, "dynamic_byte_chunking_b200", "csrc")
     assert any(f.endswith(".cu") for f in os.listdir(csrc))
+
+
+def test_comment_edits_keep_the_source_hash():
+    code = "int f(int x) {\n    return x + 1;   // add one\n}\n"
+    same = "// a new comment\nint f(int x) {\n    /* note */ return x + 1;\n}\n"
+    other = "int f(int x) {\n    return x + 2;\n}\n"
+    assert bench.strip_comments(code) == bench.strip_comments(same)
+    assert bench.strip_comments(code) != bench.strip_comments(other)
+    # string literals keep their slashes
+    assert '"a // b"' in bench.strip_comments('asm("a // b");\n')
