@@ -156,7 +156,7 @@ def cpu_baseline(w, min_seconds=10.0):
 
 def strip_comments(text):
     """Kernel source without its comments: whole-line // comments, trailing // comments on lines
-    without string literals, and /* */ blocks; blank lines dropped, trailing blanks trimmed."""
+    without string literals, and /* */ blocks; blank lines dropped, runs of blanks collapsed."""
     import re
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     out = []
@@ -165,7 +165,7 @@ def strip_comments(text):
             continue
         if '"' not in line:
             line = re.sub(r"\s*//.*$", "", line)
-        line = line.rstrip()
+        line = " ".join(line.split())
         if line:
             out.append(line)
     return "\n".join(out)
