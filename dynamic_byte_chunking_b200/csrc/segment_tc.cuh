@@ -2,7 +2,8 @@
 // Included by coding_rate.cu, which holds the segment table, the tcgen05
 // Gram and the float64 first-segment kernel this path shares.
 //
-// Per segment s (rows X_s, start state M_s = I + P_s):
+// d in {128, 512} (register-panel path), per segment s (rows X_s, start
+// state M_s = I + P_s):
 //   factor: panel Cholesky of [P_s ; I] with the identity implicit; the
 //           appended block becomes B = L_s^{-T} (L_s L_s^T = M_s);
 //   ainv:   A_s = B B^T = M_s^{-1}, stored as three bf16 pieces (hi, mid, lo)
@@ -16,6 +17,9 @@
 // G'_s = c X_s M_s^{-1} X_s^T is the in-segment Gram in the frame whitened
 // by the segment's start state, so its Cholesky diagonal is the per-position
 // Schur complement 1 + c h_t^T M_{t-1}^{-1} h_t (matrix determinant lemma).
+// d = 256 (bf16) takes the TMEM path at the end of this file instead: the
+// factor kernel keeps B = L_s^{-T} only, Y = sqrt(c) X_s B is formed on
+// tcgen05 and the in-segment Cholesky factors I + Y Y^T.
 #pragma once
 
 #include "panel_chol.cuh"
@@ -560,9 +564,9 @@ dbc_status run_tc(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, 
 }
 
 // ================================================================ d = 256: TMEM-resident factorizations
-// Segments of at most 256 positions: the start state's factorization and
-// inverse (FACTOR) and the in-segment Cholesky (INSEG) each run inside one
-// SM's tensor memory.
+// Segments of at most 256 positions: the start state's factorization with its
+// inverse factor B = L^{-T} (FACTOR) and the in-segment Cholesky (INSEG) each
+// run inside one SM's tensor memory; the whitening Y = sqrt(c) X B in between.
 constexpr int kLmaxTmem = 256;
 
 struct Layout3 {
