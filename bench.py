@@ -237,6 +237,30 @@ def write_traffic(csv_path):
     print(json.dumps(out))
 
 
+def stage_rooflines(avg_ms, N, d, rows, K, nb, pk, src):
+    """Achieved / peak of every stage of the step from its event-timed average duration.
+
+    Algorithmic work per call: coding rate 4 d^2 N flop (the rank-1 recursion: 2 d^2 for the solve and
+    2 d^2 for the update per position) against the bf16 tensor peak; Top-K, gather and upsample their
+    compulsory HBM bytes (read inputs once, write outputs once) against the HBM copy bandwidth."""
+    flops_cr = 4.0 * d * d * N
+    tf = pk.get("bf16_tflops", 1590.0)
+    hbm = pk.get("hbm_gbs", 6650.0)
+    out = {}
+    a = flops_cr / (avg_ms[0] * 1e-3) / 1e12
+    out["chunk_coding_rate"] = {"bound": "tensor", "achieved": a, "peak": tf, "unit": "TFLOP/s", "frac": a / tf,
+                                "algorithmic": f"4*d^2*N = {flops_cr:.4g} flop per call",
+                                "peak_source": src + " bf16 (burst)"}
+    by = {"chunk_topk_select": N * 4 + rows * K * 8 + (rows + 1) * 8,          # read dR, write idx
+          "chunk_gather": 2 * rows * K * d * 2,                                 # read + write chunk rows
+          "chunk_upsample": N * d * 2 + rows * K * d * 2 + nb * d * d * 2 + N * d * 4}   # H, G, W in; S out
+    for i, st in enumerate(["chunk_topk_select", "chunk_gather", "chunk_upsample"], start=1):
+        g = by[st] / (avg_ms[i] * 1e-3) / 1e9
+        out[st] = {"bound": "hbm", "achieved": g, "peak": hbm, "unit": "GB/s", "frac": g / hbm,
+                   "algorithmic": f"{by[st]} bytes per call", "peak_source": src}
+    return out
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -332,6 +356,21 @@ def run_rows(args):
             emit("NEXT-2 streaming coding rate (blocks of 256)", fam, ms, positions_per_s=N / (ms * 1e-3),
                  blocks=len(blocks), us_per_block=ms * 1e3 / len(blocks), tflops=fl / (ms * 1e-3) / 1e12)
             del blocks, state, dRs, wss
+        if w.dtype == "bf16":
+            # NEXT-4: the encoder's Canon layer (causal depthwise conv, k = 4) alone and chained with the chunker
+            gen = np.random.default_rng(11)
+            wc = bf(workloads.bf16_bits((gen.standard_normal((d, 4)) * 0.5).astype(np.float32)))
+            bc = bf(workloads.bf16_bits((gen.standard_normal(d) * 0.02).astype(np.float32)))
+            Hc = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
+            ms = _time(lambda: dbc.canon_conv1d(Hx, wc, bc, offsets=o, T=T, residual=True, out=Hc), args.reps, flush,
+                       stream)
+            by = 2 * N * d * 2
+            emit("NEXT-4 Canon conv (k=4)", fam, ms, gbs=by / (ms * 1e-3) / 1e9, frac_hbm=by / (ms * 1e-3) / 1e9 / hbm)
+            if d in (64, 128, 256, 512):
+                ms = _time(lambda: dbc.chunk_coding_rate_canon(Hx, wc, w.eps2, bc, offsets=o, T=T, residual=True,
+                                                               Hc=Hc, dR=dR, workspace=ws), args.reps, flush, stream)
+                emit("NEXT-4 Canon conv + coding rate", fam, ms, positions_per_s=N / (ms * 1e-3))
+            del Hc
         Kt = torch.from_numpy(w.K).to(dev)
         total = int(np.minimum(w.K, w.lengths).sum())
         idx = torch.empty(total, dtype=torch.int64, device=dev)
@@ -523,61 +562,85 @@ def main():
     ms_per_step = total_max / args.steps
     value = N * world / (ms_per_step * 1e-3)
 
-    # ---- roofline of the dominant stage (the coding-rate call)
+    # ---- roofline of every stage, and of the dominant one (the coding-rate call)
     pk, src = peaks()
     avg = per_stage / args.steps          # ms per call
+    stage_roof = stage_rooflines(avg, N, d, rows, K, nb, pk, src)
     dom = int(np.argmax(avg))
-    flops_cr = 4.0 * d * d * N            # rank-1 recursion: 2d^2 (solve) + 2d^2 (update) per position
-    bytes_stage = [N * d * 2 + N * 4,                       # dR: read H, write dR
-                   N * 4 + rows * K * 8 + (rows + 1) * 8,   # Top-K: read dR, write idx
-                   2 * rows * K * d * 2,                    # gather: read + write chunk rows
-                   N * d * 2 + rows * K * d * 2 + nb * d * d * 2 + N * d * 4]  # upsample
-    if dom == 0:
-        achieved = flops_cr / (avg[0] * 1e-3) / 1e12
-        peak = pk.get("bf16_tflops_sustained", 1400.0)
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": stored_traffic(stages[0]), "kernel": stages[0],
-                "algorithmic": f"4*d^2*N = {flops_cr:.3e} flop per call", "peak_source": src + " sustained bf16"}
-    else:
-        achieved = bytes_stage[dom] / (avg[dom] * 1e-3) / 1e9
-        peak = pk.get("hbm_gbs", 6650.0)
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": stored_traffic(stages[dom]), "kernel": stages[dom],
-                "algorithmic": f"{bytes_stage[dom]} bytes per call",
-                "peak_source": src}
+    roof = dict(stage_roof[stages[dom]])
+    roof["traffic"] = stored_traffic(stages[dom])
+    roof["kernel"] = stages[dom]
+    # the metric's own definition: positions / (coding rate + Top-K + gather)
+    t_chunk = float(avg[0] + avg[1] + avg[2])
+    value_chunk = N * world / (t_chunk * 1e-3)
 
-    # ---- end to end through host buffers
+    # ---- end to end through host buffers: every step copies its H from pinned host memory to the
+    # device, runs the path through the API and reads (idx, Z, S) back into pinned host memory.  Steps
+    # alternate between two lanes, each with its own stream and buffers, so one step's device-to-host
+    # copies overlap the next step's host-to-device copy and compute (full-duplex copy engines).
     e2e = None
     if args.e2e_steps > 0:
-        out_idx = torch.empty(rows * K, dtype=torch.int64).pin_memory()
-        out_Z = torch.empty(rows * K, d, dtype=torch.bfloat16).pin_memory()
-        out_S = torch.empty(N, d, dtype=torch.float32).pin_memory()
-        Hdev = torch.empty(rows, T, d, dtype=torch.bfloat16, device=dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for _ in range(2):
-            Hdev.copy_(H_host.view(rows, T, d), non_blocking=True)
-            step(Hdev)
+        class Lane:
+            def __init__(self):
+                self.s = torch.cuda.Stream(device=dev)
+                self.H = torch.empty(rows, T, d, dtype=torch.bfloat16, device=dev)
+                self.dR = torch.empty(N, dtype=torch.float32, device=dev)
+                self.idx = torch.empty(rows * K, dtype=torch.int64, device=dev)
+                self.io = torch.empty(rows + 1, dtype=torch.int64, device=dev)
+                self.Z = torch.empty(rows * K, d, dtype=torch.bfloat16, device=dev)
+                self.S = torch.empty(N, d, dtype=torch.float32, device=dev)
+                self.ws_cr = torch.empty_like(ws_cr)
+                self.ws_up = torch.empty_like(ws_up)
+                self.o_idx = torch.empty(rows * K, dtype=torch.int64).pin_memory()
+                self.o_Z = torch.empty(rows * K, d, dtype=torch.bfloat16).pin_memory()
+                self.o_S = torch.empty(N, d, dtype=torch.float32).pin_memory()
+
+            def step(self):
+                with torch.cuda.stream(self.s):
+                    flush.zero_()
+                    self.H.copy_(H_host.view(rows, T, d), non_blocking=True)
+                    dbc.chunk_coding_rate(self.H, w.eps2, dR=self.dR, workspace=self.ws_cr, dev_status=st,
+                                          stream=self.s)
+                    dbc.chunk_topk_select(self.dR, K, rows=rows, T=T, idx=self.idx, idx_offsets=self.io,
+                                          dev_status=st, stream=self.s)
+                    dbc.chunk_gather(self.H, self.idx, self.io, rows=rows, T=T, total=rows * K, Z=self.Z,
+                                     dev_status=st, stream=self.s)
+                    dbc.chunk_upsample(self.Z, self.H, self.idx, self.io, Wb, rows=rows, T=T, S=self.S,
+                                       workspace=self.ws_up, dev_status=st, stream=self.s)
+                    self.o_idx.copy_(self.idx, non_blocking=True)
+                    self.o_Z.copy_(self.Z, non_blocking=True)
+                    self.o_S.copy_(self.S, non_blocking=True)
+
+        lanes = [Lane(), Lane()]
         torch.cuda.synchronize()
-        tot = 0.0
-        for _ in range(args.e2e_steps):
-            flush.zero_()
-            e0.record(stream)
-            Hdev.copy_(H_host.view(rows, T, d), non_blocking=True)
-            step(Hdev)
-            out_idx.copy_(idx, non_blocking=True)
-            out_Z.copy_(Z, non_blocking=True)
-            out_S.copy_(S, non_blocking=True)
-            e1.record(stream)
-            e1.synchronize()
-            tot += e0.elapsed_time(e1)
-        te = torch.tensor([tot], dtype=torch.float64, device=dev)
+        for k in range(4):                    # warm-up of both lanes
+            lanes[k % 2].step()
+        torch.cuda.synchronize()
+        main_s = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main_s)
+        for ln in lanes:
+            ln.s.wait_event(e0)
+        for k in range(args.e2e_steps):
+            lanes[k % 2].step()
+        for ln in lanes:
+            ev = torch.cuda.Event()
+            ev.record(ln.s)
+            main_s.wait_event(ev)
+        e1.record(main_s)
+        e1.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
         if pg:
             pg.all_reduce(te, op=pg.ReduceOp.MAX)
         ms_e2e = float(te.item()) / args.e2e_steps
+        ln = lanes[0]
         e2e = {"value": N * world / (ms_e2e * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(H_host.numel() * 2),
-               "d2h_bytes_per_step": int(out_idx.numel() * 8 + out_Z.numel() * 2 + out_S.numel() * 4),
-               "ms_per_step": ms_e2e}
+               "d2h_bytes_per_step": int(ln.o_idx.numel() * 8 + ln.o_Z.numel() * 2 + ln.o_S.numel() * 4),
+               "ms_per_step": ms_e2e,
+               "pipelining": "two lanes (streams) alternate steps: device-to-host copies of one step overlap the "
+                             "next step's host-to-device copy and compute"}
+        del lanes
 
     torch.cuda.synchronize()
     check_status("after the timed steps")
@@ -595,6 +658,9 @@ def main():
                            "l2": "flushed by a 256 MB write before every timed step",
                            "step": " -> ".join(stages)},
                 "stage_ms": {s: float(a) for s, a in zip(stages, avg)},
+                "value_chunk": {"value": value_chunk, "unit": UNIT, "ms": t_chunk,
+                                "definition": "positions / (chunk_coding_rate + chunk_topk_select + chunk_gather)"},
+                "stage_roofline": stage_roof,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
                 "clocks": clocks}
         print(json.dumps(line), flush=True)

@@ -3,9 +3,11 @@
 chunk_upsample_noalloc serves callers that cannot give the library device
 scratch (a server whose device memory is all owned by its own pool, a plugin
 that receives only its inputs and outputs).  Its scratch is a static device
-array inside libdbc.so.  These checks call it through the C ABI, twice in a
-row with different inputs (the array keeps the previous call's contents), and
-compare with chunk_upsample at the upsampling tolerance of the parity tests.
+array inside libdbc.so.  These checks call it several times in a row with
+different inputs, the sizes going large, small, large (the array keeps the
+previous call's contents), through the C ABI and once through the Python
+binding, and compare with chunk_upsample at the upsampling tolerance of the
+parity tests.
 This file is collected last on purpose; it passes alone or after the others.
 """
 import ctypes
@@ -50,13 +52,15 @@ def _call_noalloc(L, G, H, offs_d, T, N, d_g, d_l, idx, io, rows, W, nbins, mode
                                     S.data_ptr(), st.data_ptr(), s)
 
 
-@pytest.mark.parametrize("mode", [0, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2])
 def test_noalloc_matches_workspace_entry_point_twice(mode):
     import torch
     import dynamic_byte_chunking_b200 as dbc
     L = dbc.lib()
-    cases = [_case(1, [1, 700, 64, 2000, 33]), _case(2, [4096, 5, 900])]   # different sizes back to back
-    for offs, idx, io, H, G, W in cases:
+    # large, small, large: the small call runs over scratch that a larger call left behind, and the last
+    # call over what the small one left; the middle call goes through the Python binding
+    cases = [_case(2, [4096, 5, 900]), _case(1, [1, 700, 64, 33]), _case(3, [2000, 3000, 17, 1200])]
+    for i, (offs, idx, io, H, G, W) in enumerate(cases):
         rows, N, T = len(offs) - 1, int(offs[-1]), int(np.diff(offs).max())
         nbins, d_g, d_l = W.shape
         Hd, Gd, Wd = _dev_bf16(H), _dev_bf16(G), _dev_bf16(W)
@@ -64,11 +68,15 @@ def test_noalloc_matches_workspace_entry_point_twice(mode):
         ref = dbc.chunk_upsample(Gd, Hd, idd, iod, Wd, rows=rows, T=T, offsets=od, mode=mode)
         S = torch.full((N, d_l), float("nan"), dtype=torch.float32, device="cuda")
         st = torch.zeros(1, dtype=torch.int32, device="cuda")
-        rc = _call_noalloc(L, Gd, Hd, od, T, N, d_g, d_l, idd, iod, rows, Wd, nbins, mode, S, st)
-        assert rc == 0, dbc.status_string(rc)
+        if i == 1:
+            dbc.chunk_upsample_noalloc(Gd, Hd, idd, iod, Wd, rows=rows, T=T, offsets=od, mode=mode, S=S,
+                                       dev_status=st)
+        else:
+            rc = _call_noalloc(L, Gd, Hd, od, T, N, d_g, d_l, idd, iod, rows, Wd, nbins, mode, S, st)
+            assert rc == 0, dbc.status_string(rc)
         torch.cuda.synchronize()
         assert st.item() == 0
-        check_close_rows(S.cpu().numpy(), ref.cpu().numpy(), f"noalloc-m{mode}")
+        check_close_rows(S.cpu().numpy(), ref.cpu().numpy(), f"noalloc-m{mode}-{i}")
 
 
 def test_noalloc_rejects_sizes_above_its_scratch():
