@@ -17,9 +17,10 @@
 // G'_s = c X_s M_s^{-1} X_s^T is the in-segment Gram in the frame whitened
 // by the segment's start state, so its Cholesky diagonal is the per-position
 // Schur complement 1 + c h_t^T M_{t-1}^{-1} h_t (matrix determinant lemma).
-// d = 256 (bf16) takes the TMEM path at the end of this file instead: the
-// factor kernel keeps B = L_s^{-T} only, Y = sqrt(c) X_s B is formed on
-// tcgen05 and the in-segment Cholesky factors I + Y Y^T.
+// d = 256 (bf16) takes the TMEM path at the end of this file instead: a fused
+// TMA-fed Gram + float64 prefix kernel gives every segment's start state, the
+// factor kernel keeps B = L_s^{-T} only, and the in-segment kernel forms
+// Y = sqrt(c) X_s B on tcgen05 itself and factors I + Y Y^T.
 #pragma once
 
 #include "panel_chol.cuh"
@@ -312,138 +313,6 @@ __global__ void __launch_bounds__(128, 1) vgemm_kernel(const __nv_bfloat16 *__re
     if (warp == 0) tc::tmem_dealloc(tbase, D);
 }
 
-// Y = sqrt(c) X_s B_s for a whole segment of up to 256 positions in one CTA
-// (d = 256): both 128-row blocks accumulate in TMEM (columns 0 and 256), so
-// each piece of B_s is read once per segment.  B_s = L_s^{-T} is upper
-// triangular and was stored per 16-column panel for the rows above the
-// panel's end only; the loads zero-fill the rest.  Y is written as three bf16
-// pieces through shared memory in whole 128-byte row segments.
-struct YSegCfg {
-    static constexpr int NS = 3;
-    static constexpr uint32_t X_BYTES = 2 * 128 * 128;         // 256 positions x 64 K (K-major)
-    static constexpr uint32_t STAGE = X_BYTES + 4 * 8192;      // + 64 K x 256 columns of B (MN-major)
-    static constexpr size_t SMEM = NS * STAGE + 1024;
-};
-static_assert(YSegCfg::NS * YSegCfg::STAGE >= 3u * 256u * 144u, "epilogue staging must fit in the stages");
-
-__global__ void __launch_bounds__(256, 1) ygemm_seg_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
-                                                           const __nv_bfloat16 *__restrict__ Bscr,
-                                                           __nv_bfloat16 *Y3, int64_t N, float scale, int32_t *st) {
-    constexpr int D = 256, KC = D / 64, NCH = 3 * KC, NS = YSegCfg::NS;
-    extern __shared__ uint8_t smraw[];
-    __shared__ uint64_t mbar[NS];
-    __shared__ uint32_t tmem_base;
-    const int s = blockIdx.x;
-    if (s >= *S.nseg) return;
-    const int len = S.len[s];
-    const int64_t start = S.start[s];
-    const int nblk = len > 128 ? 2 : 1;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
-    if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
-    if (tid == 0) {
-        for (int i = 0; i < NS; ++i) tc::mbar_init(&mbar[i], 1);
-        tc::fence_mbar_init();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tbase = tmem_base;
-    const __nv_bfloat16 *Xs = H + start * D;
-    const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
-    auto load = [&](int c, uint32_t sa) {
-        const int p = c / KC, kc = c % KC;
-        for (int e = tid; e < 256 * 8; e += 256) {            // X: 256 positions x 8 units of 8 K
-            const int r = e >> 3, ch = e & 7;
-            const bool in = r < len;
-            const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
-            tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + kc * 64 + ch * 8, in ? 16u : 0u);
-        }
-        const uint32_t sb = sa + YSegCfg::X_BYTES;
-        for (int e = tid; e < 64 * 32; e += 256) {            // B: 64 K rows x 32 units of 8 columns
-            const int k = e >> 5, n8 = e & 31;
-            const int kr = kc * 64 + k;
-            const bool nz = kr < (n8 >> 1) * 16 + 16;         // stored rows of the columns' panel
-            tc::cp_async16(sb + tc::mnmajor_off(n8 * 8, k, 8192),
-                           Bseg + (size_t)p * D * D + (size_t)(nz ? kr : 0) * D + n8 * 8, nz ? 16u : 0u);
-        }
-    };
-    constexpr uint32_t idesc = tc::idesc_bf16(128, 256, false, true);
-    bool ok = true;
-    for (int c = 0; c < NS - 1; ++c) {
-        load(c, base + (uint32_t)c * YSegCfg::STAGE);
-        tc::cp_async_commit();
-    }
-    for (int c = 0; c < NCH; ++c) {
-        const int cn = c + NS - 1;
-        if (cn < NCH) {
-            if (cn >= NS) ok &= tc::mbar_wait(&mbar[cn % NS], (uint32_t)((cn / NS) - 1) & 1u, st);
-            load(cn, base + (uint32_t)(cn % NS) * YSegCfg::STAGE);
-        }
-        tc::cp_async_commit();
-        tc::cp_async_wait<NS - 1>();
-        tc::fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t sa = base + (uint32_t)(c % NS) * YSegCfg::STAGE, sb = sa + YSegCfg::X_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bd = tc::sdesc(sb + kk * 2048, 8192, 1024);
-                for (int b = 0; b < nblk; ++b)
-                    tc::mma_bf16(tbase + (uint32_t)(b * 256), tc::sdesc(sa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
-                                 bd, idesc, (c > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc::mma_commit(&mbar[c % NS]);
-        }
-        __syncthreads();
-    }
-    ok &= tc::mbar_wait(&mbar[(NCH - 1) % NS], (uint32_t)((NCH - 1) / NS) & 1u, st);
-    ok = __syncthreads_and(ok) != 0;
-    tc::fence_after_sync();
-    if (ok) {
-        tc::cp_async_wait<0>();
-        __syncthreads();
-        uint8_t *stg = smraw + (base - tc::smem_u32(smraw));
-        constexpr int RS = 144;
-        __nv_bfloat16 *yb = Y3 + (size_t)start * D;
-        // warps 0-3 read the first row block's lanes, warps 4-7 the second's (TMEM columns + 256)
-        const int b = warp >> 2, lg = warp & 3;
-        const int row = b * 128 + lg * 32 + lane;
-#pragma unroll 1
-        for (int cb = 0; cb < D; cb += 64) {
-            if (b < nblk) {                                       // warp-uniform
-#pragma unroll 1
-                for (int j = 0; j < 4; ++j) {
-                    float v[16];
-                    tc::tmem_ld16(tbase + ((uint32_t)(lg * 32) << 16) + (uint32_t)(b * 256 + cb + 16 * j), v);
-                    __align__(16) __nv_bfloat16 h[16], m[16], l[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) split3(scale * v[i], h[i], m[i], l[i]);
-#pragma unroll
-                    for (int p = 0; p < 3; ++p) {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(p == 0 ? h : (p == 1 ? m : l));
-                        uint4 *d = reinterpret_cast<uint4 *>(stg + (size_t)(p * 256 + row) * RS + j * 32);
-                        d[0] = src[0];
-                        d[1] = src[1];
-                    }
-                }
-            }
-            __syncthreads();
-            for (int e = tid; e < 3 * 256 * 8; e += 256) {
-                const int pr = e >> 3, ch = e & 7, p = pr >> 8, r = pr & 255;
-                if (r < len)
-                    *reinterpret_cast<uint4 *>(yb + (size_t)p * N * D + (size_t)r * D + cb + ch * 8) =
-                        *reinterpret_cast<const uint4 *>(stg + (size_t)pr * RS + ch * 16);
-            }
-            __syncthreads();
-        }
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tbase, 512);
-}
-
 struct KCfg {
     static constexpr int NS = 4;
     static constexpr uint32_t STAGE = 128 * 128 + 128 * 128;
@@ -573,7 +442,6 @@ struct Layout3 {
     Segs segs;
     float *P;               // per segment: [D][D] Gram -> c-scaled prefix
     __nv_bfloat16 *Bscr;    // per segment: [3][D][D] pieces of B = L^{-T} (rows below a panel unstored)
-    __nv_bfloat16 *Y3;      // [3][N][D] pieces of Y = sqrt(c) X_s B_s
     size_t bytes;
 };
 
@@ -591,7 +459,6 @@ inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d, int64_t ns_g
     L.segs.nseg = c.take<int32_t>(1);
     L.P = c.take<float>((size_t)ns * d * d);
     L.Bscr = c.take<__nv_bfloat16>((size_t)ns * 3 * d * d);
-    L.Y3 = c.take<__nv_bfloat16>((size_t)3 * N * d + 8);
     L.bytes = c.off;
     return L;
 }
@@ -600,9 +467,36 @@ inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d, int64_t ns_g
 }  // namespace dbc
 
 #include "tmem_chol.cuh"
+#include "gram_prefix.cuh"
+#include "tma_host.cuh"
 
 namespace dbc {
 namespace cr {
+
+// P_s = c (state + the row's earlier segment Grams) for every segment, through the fused TMA-fed
+// Gram + float64 prefix kernel (one CTA per row and 128 x TN tile).  Returns false (nothing
+// launched) when the row count and lengths favour the segment-parallel Gram and prefix kernels,
+// or when no tensor map can be encoded.
+inline bool launch_gram_prefix(const __nv_bfloat16 *H, int64_t N, int64_t rows, int64_t ns, const Segs &segs,
+                               float *P, double *state, double c, int32_t *st, cudaStream_t stream) {
+    const int sms = num_sms();
+    // few long rows leave most SMs idle in a per-row walk
+    if (rows * 6 < sms && ns > rows * 128) return false;
+    if (rows * 6 > INT32_MAX / 2) return false;
+    CUtensorMap tm;
+    if (!tma::encode_bf16_rows(&tm, H, (uint64_t)N, 256, 64)) return false;
+    if (rows * 6 <= 2 * (int64_t)sms) {
+        using C = GramPrefixCfg<64>;
+        cudaFuncSetAttribute(gram_prefix_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+        gram_prefix_kernel<64><<<(unsigned)(rows * C::TILES), C::NT, C::SMEM, stream>>>(tm, segs, rows, P, state, c, st);
+    } else {
+        using C = GramPrefixCfg<128>;
+        cudaFuncSetAttribute(gram_prefix_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+        gram_prefix_kernel<128><<<(unsigned)(rows * C::TILES), C::NT, C::SMEM, stream>>>(tm, segs, rows, P, state, c,
+                                                                                        st);
+    }
+    return true;
+}
 
 inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N,
                            float eps2, float *dR, const Layout3 &L, int32_t *st, cudaStream_t stream) {
@@ -611,18 +505,20 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     const int64_t ns = nseg_upper(rows, N, kLmaxTmem);
     const int sms = num_sms();
     seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kLmaxTmem, L.segs, st);
-    launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
-    prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
-        L.segs, L.P, D, c, (size_t)D * D);
+    const bool fused = launch_gram_prefix(H, N, rows, ns, L.segs, L.P, nullptr, c, st, stream);
+    if (!fused) {
+        launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
+        prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
+            L.segs, L.P, D, c, (size_t)D * D);
+    }
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, dR, st);
-    cudaFuncSetAttribute(ygemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)YSegCfg::SMEM);
-    ygemm_seg_kernel<<<(unsigned)ns, 256, YSegCfg::SMEM, stream>>>(H, L.segs, L.Bscr, L.Y3, N, (float)std::sqrt(c),
-                                                                   st);
-    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, nullptr, L.Y3, N, dR, st);
-    count_launches(6);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, (float)c,
+                                                                         dR, st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, L.Bscr, H, N, (float)c, dR,
+                                                                          st);
+    count_launches(fused ? 4 : 5);
     return launch_status();
 }
 
@@ -706,18 +602,20 @@ inline dbc_status run_tmem_stream(const __nv_bfloat16 *H, int64_t streams, int64
     const int sms = num_sms();
     const int tgrid = (int)std::max<int64_t>(1, std::min<int64_t>((ns + 255) / 256, (int64_t)sms * 4));
     stream_seg_table_kernel<<<tgrid, 256, 0, stream>>>(streams, n, t0, k1, cnt, L.segs);
-    launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
-    prefix_stream_kernel<<<dim3((unsigned)streams, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
-        L.segs, L.P, state, D, c);
+    const bool fused = launch_gram_prefix(H, N, streams, ns, L.segs, L.P, state, c, st, stream);
+    if (!fused) {
+        launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
+        prefix_stream_kernel<<<dim3((unsigned)streams, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
+            L.segs, L.P, state, D, c);
+    }
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, dR, st);
-    cudaFuncSetAttribute(ygemm_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)YSegCfg::SMEM);
-    ygemm_seg_kernel<<<(unsigned)ns, 256, YSegCfg::SMEM, stream>>>(H, L.segs, L.Bscr, L.Y3, N, (float)std::sqrt(c),
-                                                                   st);
-    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, nullptr, L.Y3, N, dR, st);
-    count_launches(6);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, (float)c,
+                                                                         dR, st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, L.Bscr, H, N, (float)c, dR,
+                                                                          st);
+    count_launches(fused ? 4 : 5);
     return launch_status();
 }
 

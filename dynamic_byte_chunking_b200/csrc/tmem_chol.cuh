@@ -36,8 +36,13 @@ struct TmemChol {
     static constexpr int NT = 256;
     static constexpr uint32_t PIECE = 256 * 128;          // 256-row x 64-K bf16 tile
     static constexpr uint32_t PANEL = 3 * PIECE;          // staged panel (three pieces)
-    static constexpr uint32_t GSTAGE = 3 * PIECE;         // G' GEMM stage: the three pieces of Y, 64 K
-    static constexpr uint32_t REGION = (2 * GSTAGE > PANEL) ? 2 * GSTAGE : PANEL;
+    // in-segment Gram: the pieces of Y_c (3 x PIECE), then two operand stages of X (256 x 64 K,
+    // K-major) and the three pieces of a 64 x 64 block of B (MN-major)
+    static constexpr uint32_t YX_BYTES = 2 * 128 * 128;
+    static constexpr uint32_t YSTAGE = YX_BYTES + 3 * 8192;
+    static constexpr uint32_t YSTAGE0 = 3 * PIECE;
+    static constexpr uint32_t YREGION = YSTAGE0 + 2 * YSTAGE;
+    static constexpr uint32_t REGION = (YREGION > 2 * PANEL) ? YREGION : 2 * PANEL;
     static constexpr size_t SMEM = REGION + 1024;
 };
 
@@ -151,11 +156,12 @@ __device__ __forceinline__ uint32_t idesc_neg(int N) { return tc::idesc_bf16(128
 
 template <bool FACTOR>
 __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
-    Segs S, const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr, const __nv_bfloat16 *__restrict__ Y3,
-    int64_t N, float *dR, int32_t *st) {
+    Segs S, const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr, const __nv_bfloat16 *__restrict__ Hx,
+    int64_t N, float c_rate, float *dR, int32_t *st) {
     constexpr int D = 256;
     extern __shared__ uint8_t smraw[];
-    __shared__ uint64_t mbar[2];
+    // [0], [1] panel MMA groups; [2] the final drain; [3], [4] Y operand stages consumed; [5] Y chunk done
+    __shared__ uint64_t mbar[6];
     __shared__ uint32_t tmem_base;
     __shared__ __align__(16) float s_LdT[16][16];   // factored 16 x 16 diagonal block, column-major
     __shared__ __align__(16) float s_rl[16];        // 1 / L_kk of the diagonal block
@@ -165,8 +171,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     const uint32_t region = (tc::smem_u32(smraw) + 1023u) & ~1023u;
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
-        tc::mbar_init(&mbar[0], 1);
-        tc::mbar_init(&mbar[1], 1);
+        for (int i = 0; i < 6; ++i) tc::mbar_init(&mbar[i], 1);
         tc::fence_mbar_init();
     }
     tc::fence_before_sync();
@@ -175,6 +180,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     const uint32_t tbase = tmem_base;
     const uint32_t trow = tbase + ((uint32_t)lb << 16) + (uint32_t)(blk * 256);
     uint32_t ph0 = 0, ph1 = 0;      // mbarrier phases (uniform across threads)
+    uint32_t phs[2] = {0, 0}, phy = 0;
     bool ok = true;
     const int nseg = *S.nseg;
 
@@ -209,57 +215,119 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             }
             tc::tmem_wait_st();
         } else {
-            // G' = Y Y^T: per 64-feature chunk the three pieces of the segment's Y rows, six piece
-            // products; rows 0..127 only need columns 0..127 (the lower triangle); two stages
-            constexpr int NCH = D / 64;
-            auto load = [&](int c, uint32_t sb) {
-                for (int e = tid; e < 3 * 256 * 8; e += TmemChol::NT) {
-                    const int p = e >> 11, r = (e >> 3) & 255, ch = e & 7;
+            // G' = Y Y^T with the whitened rows Y = sqrt(c) X_s B_s formed here, 64 features at a
+            // time: Y_c = X_s B_s[:, chunk c] accumulates in the TMEM columns 128..255 (free in this
+            // mode: the first row block only uses its lower triangle), over the K chunks k <= c (B
+            // is upper triangular) with X and the three pieces of B streamed through two cp.async
+            // stages; Y_c is then split into three bf16 pieces in shared memory and G' += Y_c Y_c^T
+            // (six piece products) is issued while the next chunk's Y MMAs follow in the pipe.
+            const __nv_bfloat16 *Xs = Hx + start * D;
+            const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
+            const uint32_t yp = region;                                    // Y_c pieces, K-major
+            auto load = [&](int pi, uint32_t sa) {
+                int c = 0, k = pi;
+                while (k > c) { k -= c + 1; ++c; }                         // pair pi -> (chunk c, K chunk k)
+                for (int e = tid; e < 256 * 8; e += TmemChol::NT) {        // X: 256 positions x 64 K
+                    const int r = e >> 3, ch = e & 7;
                     const bool in = r < len;
-                    const __nv_bfloat16 *gy = Y3 + (size_t)p * N * D + (size_t)(start + (in ? r : 0)) * D + c * 64 + ch * 8;
-                    tc::cp_async16(sb + (uint32_t)p * TmemChol::PIECE + tc::kmajor_off(r, ch * 8), gy, in ? 16u : 0u);
+                    const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
+                    tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + k * 64 + ch * 8, in ? 16u : 0u);
+                }
+                const uint32_t sb = sa + TmemChol::YX_BYTES;
+                for (int e = tid; e < 3 * 64 * 8; e += TmemChol::NT) {     // B: 3 pieces x 64 K x 64 N
+                    const int p = e >> 9, kr = (e >> 3) & 63, n8 = e & 7;
+                    const int krow = k * 64 + kr, col = c * 64 + n8 * 8;
+                    const bool nz = krow < (col >> 4) * 16 + 16;             // stored rows of the columns' panel
+                    tc::cp_async16(sb + (uint32_t)p * 8192 + tc::mnmajor_off(n8 * 8, kr, 8192),
+                                   Bseg + (size_t)p * D * D + (size_t)(nz ? krow : 0) * D + col, nz ? 16u : 0u);
                 }
             };
+            constexpr int NPAIR = 10;                                      // (c, k) with k <= c < 4
+            constexpr uint32_t idy = tc::idesc_bf16(128, 64, false, true);
             constexpr uint32_t idg0 = tc::idesc_bf16(128, 128, false, false);
             constexpr uint32_t idg1 = tc::idesc_bf16(128, 256, false, false);
-            load(0, region);
+            const float sc = sqrtf(c_rate);
+            load(0, region + TmemChol::YSTAGE0);
             tc::cp_async_commit();
-            for (int c = 0; c < NCH; ++c) {
-                if (c + 1 < NCH) {
-                    if (c >= 1) {     // stage (c+1)%2 was read by the MMAs of chunk c-1
-                        ok &= tc::mbar_wait(&mbar[(c + 1) & 1], ((c + 1) & 1) ? ph1 : ph0, st);
-                        if ((c + 1) & 1) ph1 ^= 1; else ph0 ^= 1;
+            for (int pi = 0; pi < NPAIR; ++pi) {
+                int c = 0, k = pi;
+                while (k > c) { k -= c + 1; ++c; }
+                if (pi + 1 < NPAIR) {
+                    const int q = (pi + 1) & 1;
+                    if (pi + 1 >= 2) {                                      // stage q was read by pair pi - 1
+                        ok &= tc::mbar_wait(&mbar[3 + q], phs[q], st);
+                        phs[q] ^= 1;
                     }
-                    load(c + 1, region + (uint32_t)((c + 1) & 1) * TmemChol::GSTAGE);
+                    load(pi + 1, region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE);
                 }
                 tc::cp_async_commit();
                 tc::cp_async_wait<1>();
                 tc::fence_async_smem();
                 __syncthreads();
+                const uint32_t sa = region + TmemChol::YSTAGE0 + (uint32_t)(pi & 1) * TmemChol::YSTAGE;
                 if (tid == 0) {
                     tc::fence_after_sync();
-                    const uint32_t sb = region + (uint32_t)(c & 1) * TmemChol::GSTAGE;
+                    const uint32_t sb = sa + TmemChol::YX_BYTES;
 #pragma unroll
-                    for (int pr = 0; pr < 6; ++pr) {
-                        const uint32_t pa = sb + (uint32_t)pair_a(pr) * TmemChol::PIECE;
-                        const uint32_t pb = sb + (uint32_t)pair_b(pr) * TmemChol::PIECE;
+                    for (int b = 0; b < 2; ++b)
 #pragma unroll
-                        for (int b = 0; b < 2; ++b)
+                        for (int p = 0; p < 3; ++p)
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                tc::mma_bf16(tbase + (uint32_t)(b * 256),
-                                             tc::sdesc(pa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
-                                             tc::sdesc(pb + kk * 32, 16, 1024), b == 0 ? idg0 : idg1,
-                                             (c > 0 || pr > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc::mma_commit(&mbar[c & 1]);
+                                tc::mma_bf16(tbase + (uint32_t)(128 + b * 64),
+                                             tc::sdesc(sa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
+                                             tc::sdesc(sb + (uint32_t)p * 8192 + kk * 2048, 8192, 1024), idy,
+                                             (k > 0 || p > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&mbar[3 + (pi & 1)]);
+                    if (k == c) tc::mma_commit(&mbar[5]);
                 }
-                __syncthreads();
+                if (k == c) {
+                    // Y_c complete (and with it every earlier MMA, so the pieces buffer is free)
+                    ok &= tc::mbar_wait(&mbar[5], phy, st);
+                    phy ^= 1;
+                    tc::fence_after_sync();
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (ok) {
+                        float a64[64];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float v16[16];
+                            tc::tmem_ld16(tbase + ((uint32_t)lb << 16) + (uint32_t)(128 + blk * 64 + q * 16), v16);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) a64[q * 16 + i] = sc * v16[i];
+                        }
+                        stage_row(yp, row, a64, nullptr, 0);
+                    }
+                    tc::fence_async_smem();
+                    tc::fence_before_sync();
+                    ok = __syncthreads_and(ok) != 0;
+                    if (!ok) break;
+                    if (tid == 0) {
+                        tc::fence_after_sync();
+#pragma unroll
+                        for (int pr = 0; pr < 6; ++pr) {
+                            const uint32_t pa = yp + (uint32_t)pair_a(pr) * TmemChol::PIECE;
+                            const uint32_t pb = yp + (uint32_t)pair_b(pr) * TmemChol::PIECE;
+#pragma unroll
+                            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    tc::mma_bf16(tbase + (uint32_t)(b * 256),
+                                                 tc::sdesc(pa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
+                                                 tc::sdesc(pb + kk * 32, 16, 1024), b == 0 ? idg0 : idg1,
+                                                 (c > 0 || pr > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                }
             }
-            // wait for the last two chunks' MMAs
-            for (int c = (NCH >= 2 ? NCH - 2 : 0); c < NCH; ++c) {
-                ok &= tc::mbar_wait(&mbar[c & 1], (c & 1) ? ph1 : ph0, st);
-                if (c & 1) ph1 ^= 1; else ph0 ^= 1;
+            if (!ok) break;
+            // G' complete; the last two stage commits are consumed so every commit has its wait
+            if (tid == 0) tc::mma_commit(&mbar[5]);
+            ok &= tc::mbar_wait(&mbar[5], phy, st);
+            phy ^= 1;
+            for (int q = 0; q < 2; ++q) {
+                ok &= tc::mbar_wait(&mbar[3 + q], phs[q], st);
+                phs[q] ^= 1;
             }
         }
         tc::fence_before_sync();
@@ -268,20 +336,71 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
 
-        // ---------------- 16-column panels
-        // Each panel: its 16 TMEM columns -> registers; the 16 x 16 diagonal block is factored by
-        // its half-warp with shuffles; every other live row solves its 16 values against it; the
-        // values are staged as three bf16 pieces and all later columns are updated by tcgen05 MMAs
-        // (negated A, six piece products, K = 16).  Two barriers and one MMA wait per panel.
+        // ---------------- 16-column panels with a one-panel look-ahead
+        // Panel j: its 16 TMEM columns -> registers; the 16 x 16 diagonal block is factored by its
+        // half-warp with shuffles; every other live row solves its 16 values against it; the values
+        // are staged as three bf16 pieces (two staging buffers, alternating) and one thread issues
+        // the negated K = 16 tcgen05 MMAs of the trailing update in two groups: the next panel's 16
+        // columns (committed to mbar[0]) and then every later column (committed to mbar[1]).  Panel
+        // j+1 waits for mbar[0] only, so the bulk of the update runs under its factorization.  In
+        // the factor mode the rows of the diagonal block must start their B entries right of the
+        // panel from zero: the other warp of their TMEM lane group resets those entries once the
+        // previous panel's bulk update has landed, while the diagonal block is being factored.
         __nv_bfloat16 *Bs = FACTOR ? Bscr + (size_t)s * 3 * D * D : nullptr;
-        for (int j0 = 0; j0 < n; j0 += 16) {
+        const int npan = (n + 15) / 16;
+        // phase bookkeeping: panel j < npan - 1 commits once to each barrier; completion k of a
+        // barrier is awaited with parity (base + k) & 1
+        const uint32_t base0 = ph0, base1 = ph1;
+        for (int j = 0; j < npan; ++j) {
+            const int j0 = 16 * j;
             const int nb = min(16, n - j0);
             const int j1 = j0 + nb;
             const int ii = row - j0;
             const bool diag = ii >= 0 && ii < 16;
+            const uint32_t R = region + (uint32_t)(j & 1) * TmemChol::PANEL;
+            if (j > 0) {
+                // the previous panel's update of these 16 columns (and every earlier MMA) has landed;
+                // a timeout is acted on at the next block-wide vote
+                ok &= tc::mbar_wait(&mbar[0], (base0 + (uint32_t)(j - 1)) & 1u, st);
+                tc::fence_after_sync();
+            }
             float v[16];
             __syncwarp();
             tc::tmem_ld16(trow + (uint32_t)j0, v);
+            const int gd = (j0 & 127) >> 5, bd = j0 >> 7;     // lane group, row block of the block rows
+            if (FACTOR && j1 < n && warp == (1 - bd) * 4 + gd) {   // warp-uniform: the reset helper
+                bool okh = true;
+                if (j > 0) {
+                    okh = tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(j - 1)) & 1u, st);   // previous bulk update
+                    tc::fence_after_sync();
+                }
+                okh = __all_sync(0xffffffffu, okh);
+                if (okh) {
+                    const int lrow = bd * 128 + gd * 32 + lane;   // row of this lane in those columns
+                    const bool zero = lrow >= j0 && lrow < j0 + 16;
+                    const uint32_t tb = tbase + ((uint32_t)(gd * 32) << 16) + (uint32_t)(bd * 256);
+#pragma unroll 1
+                    for (int c0 = j1; c0 < D; c0 += 64) {
+                        const int cnt = min(4, (D - c0) >> 4);      // warp-uniform
+                        uint32_t r4[4][16];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (q < cnt) tc::tmem_ld16_nw(tb + (uint32_t)(c0 + 16 * q), r4[q]);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (q < cnt) {
+                                float t16[16];
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) t16[i] = zero ? 0.f : __uint_as_float(r4[q][i]);
+                                tc::tmem_st16(tb + (uint32_t)(c0 + 16 * q), t16);
+                            }
+                        }
+                    }
+                    tc::tmem_wait_st();
+                }
+                ok &= okh;
+            }
             if (FACTOR && diag) {
                 // right of its diagonal a row carries B, which only receives contributions from
                 // columns at or after its own: what earlier updates left there is dropped
@@ -316,11 +435,12 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     e_mine = piv ? e : e_mine;
                 }
                 s_rl[ii] = rl_mine;
-                if (!FACTOR && ii < nb) dR[start + j0 + ii] = 0.5f * log1pf(e_mine);
+                if (!FACTOR && ii < nb && dcheck(start + j0 + ii < N, st)) dR[start + j0 + ii] = 0.5f * log1pf(e_mine);
 #pragma unroll
                 for (int c = 0; c < 16; ++c) s_LdT[c][ii] = c <= ii ? v[c] : 0.f;
             }
-            __syncthreads();
+            ok = __syncthreads_and(ok) != 0;
+            if (!ok) break;
             // rows at or above the block are finished in the in-segment mode
             const bool live = FACTOR || ii >= 16;
             if (live) {
@@ -329,9 +449,9 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 // B_ii = 1/L_ii); rows above the block carry B, rows below L
                 float rl[16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 r4 = reinterpret_cast<const float4 *>(s_rl)[j];
-                    rl[4 * j] = r4.x; rl[4 * j + 1] = r4.y; rl[4 * j + 2] = r4.z; rl[4 * j + 3] = r4.w;
+                for (int q = 0; q < 4; ++q) {
+                    const float4 r4 = reinterpret_cast<const float4 *>(s_rl)[q];
+                    rl[4 * q] = r4.x; rl[4 * q + 1] = r4.y; rl[4 * q + 2] = r4.z; rl[4 * q + 3] = r4.w;
                 }
                 const float binv = diag ? 1.f / s_LdT[ii][ii] : 0.f;      // B_ii = 1 / L_ii (IEEE)
 #pragma unroll
@@ -341,13 +461,13 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     a[m] = am;
                     const float4 *lr = reinterpret_cast<const float4 *>(&s_LdT[m][0]);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (4 * j + 3 > m) {
-                            const float4 l = lr[j];
-                            if (4 * j + 0 > m) v[4 * j + 0] = fmaf(-am, l.x, v[4 * j + 0]);
-                            if (4 * j + 1 > m) v[4 * j + 1] = fmaf(-am, l.y, v[4 * j + 1]);
-                            if (4 * j + 2 > m) v[4 * j + 2] = fmaf(-am, l.z, v[4 * j + 2]);
-                            v[4 * j + 3] = fmaf(-am, l.w, v[4 * j + 3]);
+                    for (int q = 0; q < 4; ++q) {
+                        if (4 * q + 3 > m) {
+                            const float4 l = lr[q];
+                            if (4 * q + 0 > m) v[4 * q + 0] = fmaf(-am, l.x, v[4 * q + 0]);
+                            if (4 * q + 1 > m) v[4 * q + 1] = fmaf(-am, l.y, v[4 * q + 1]);
+                            if (4 * q + 2 > m) v[4 * q + 2] = fmaf(-am, l.z, v[4 * q + 2]);
+                            v[4 * q + 3] = fmaf(-am, l.w, v[4 * q + 3]);
                         }
                     }
                 }
@@ -379,36 +499,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             if (j1 < n) {
                 // operand rows of the trailing update: L (rows >= j1), B (factor mode, rows < j1),
                 // zero (in-segment mode, rows < j1)
-                stage_row16(region, row, a);
-                // factor mode: the diagonal rows' B entries right of the panel start from zero.
-                // tcgen05.ld/st are warp-collective (.sync.aligned) and a warp may only address its
-                // lane group, so the two warps of the block rows' lane group (one per row block)
-                // read the columns past the panel and write them back, zeros for the block rows;
-                // each takes every other 32 columns, two loads in flight per wait.
-                const int gd = (j0 & 127) >> 5, bd = j0 >> 7;     // lane group, row block of the block
-                if (FACTOR && (warp & 3) == gd) {                 // warp-uniform
-                    __syncwarp();
-                    const int lrow = bd * 128 + gd * 32 + lane;   // row of this lane in those columns
-                    const bool zero = lrow >= j0 && lrow < j0 + 16;
-                    const uint32_t tb = tbase + ((uint32_t)(gd * 32) << 16) + (uint32_t)(bd * 256);
-#pragma unroll 1
-                    for (int c0 = j1 + 32 * (warp >> 2); c0 < D; c0 += 64) {
-                        const bool two = c0 + 16 < D;             // warp-uniform
-                        uint32_t r0[16], r1[16] = {};
-                        tc::tmem_ld16_nw(tb + (uint32_t)c0, r0);
-                        if (two) tc::tmem_ld16_nw(tb + (uint32_t)(c0 + 16), r1);
-                        tc::tmem_wait_ld();
-                        float t0[16], t1[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            t0[i] = zero ? 0.f : __uint_as_float(r0[i]);
-                            t1[i] = zero ? 0.f : __uint_as_float(r1[i]);
-                        }
-                        tc::tmem_st16(tb + (uint32_t)c0, t0);
-                        if (two) tc::tmem_st16(tb + (uint32_t)(c0 + 16), t1);
-                    }
-                    tc::tmem_wait_st();
-                }
+                stage_row16(R, row, a);
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
@@ -416,27 +507,45 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             if (j1 < n) {
                 if (tid == 0) {
                     tc::fence_after_sync();
+                    // the next panel's 16 columns first, then everything right of them
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        if (!FACTOR && (b + 1) * 128 <= j1) continue;
+                        issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1), R, b * 128, j1, idesc_neg(16));
+                    }
+                    tc::mma_commit(&mbar[0]);
 #pragma unroll
                     for (int b = 0; b < 2; ++b) {
                         if (!FACTOR && (b + 1) * 128 <= j1) continue;
                         // in-segment mode: the first row block only needs its lower triangle (columns < 128)
-                        const int nc = (!FACTOR && b == 0) ? 128 - j1 : 256 - j1;
-                        issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1), region, b * 128, j1, idesc_neg(nc));
+                        const int nc = ((!FACTOR && b == 0) ? 128 : 256) - j1 - 16;
+                        if (nc > 0)
+                            issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1 + 16), R, b * 128, j1 + 16,
+                                                idesc_neg(nc));
                     }
-                    tc::mma_commit(&mbar[0]);
+                    tc::mma_commit(&mbar[1]);
                 }
-                ok &= tc::mbar_wait(&mbar[0], ph0, st);
-                ph0 ^= 1;
-                tc::fence_after_sync();
-                ok = __syncthreads_and(ok) != 0;
-                if (!ok) break;
             }
         }
+        // every MMA of this segment has landed before the next segment (or the exit) reuses TMEM
+        if (ok && npan > 1) {
+            ok &= tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(npan - 2)) & 1u, st);
+            tc::fence_after_sync();
+        }
+        ph0 = (base0 + (uint32_t)(npan - 1)) & 1u;
+        ph1 = (base1 + (uint32_t)(npan - 1)) & 1u;
+        ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
 
     }
+    if (tid == 0) {
+        // MMAs still in flight (only after a timeout) finish before the tensor memory is freed
+        tc::mma_commit(&mbar[2]);
+        tc::mbar_wait(&mbar[2], 0, st);
+    }
     tc::fence_before_sync();
     __syncthreads();
+    tc::fence_after_sync();
     if (warp == 0) tc::tmem_dealloc(tbase, 512);
 }
 
