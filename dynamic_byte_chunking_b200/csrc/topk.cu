@@ -7,9 +7,10 @@
 //
 // One CTA per row: the row's dR values become order-preserving 32-bit keys
 // (in shared memory when they fit), a 4-pass 8-bit radix select finds the
-// (K-1)-th largest key v and how many keys equal to v are still needed, and
-// one ordered pass writes the selected positions, which are then already in
-// increasing order (no sort).
+// (K-1)-th largest key v and how many keys equal to v are still needed (the
+// histogram increments are aggregated per warp: the keys of a row share their
+// leading bytes), and one ordered pass writes the selected positions, which are
+// then already in increasing order (no sort).
 #include "common.cuh"
 
 namespace dbc {
@@ -102,10 +103,33 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int64_t *offsets, i
     if (tid == 0) idx_offsets[rows] = carry;
 }
 
+// Histogram increment with a warp-uniform fast path: the keys of a row share
+// their leading bytes (positive values of a narrow range), so in the early
+// passes all matching lanes of a warp usually fall into one bin, and one lane
+// adds their count; otherwise every lane adds its own (shared atomics).
+__device__ __forceinline__ void hist_add(uint32_t *hist, bool match, uint32_t bin) {
+    const unsigned active = __ballot_sync(0xffffffffu, match);
+    if (!active) return;
+    const int leader = __ffs(active) - 1;
+    const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+    const bool same = __all_sync(0xffffffffu, !match || bin == b0);
+    if (same) {
+        if ((int)(threadIdx.x & 31) == leader) atomicAdd(&hist[b0], (uint32_t)__popc(active));
+    } else if (match) {
+        atomicAdd(&hist[bin], 1u);
+    }
+}
+
+constexpr int kPerThread = 8;                         // consecutive keys per thread in the compaction
+constexpr int kTile = kThreads * kPerThread;          // keys per compaction tile
+
+// dense_K > 0: dense rows with one K for all rows, row r's indices start at
+// r * min(K, T) and this kernel writes idx_offsets; otherwise idx_offsets was
+// written by offsets_kernel.
 __global__ void __launch_bounds__(kThreads) select_kernel(const float *__restrict__ dR,
                                                           const int64_t *offsets, int64_t rows, int64_t T,
-                                                          const int64_t *Kp, int64_t Ks,
-                                                          const int64_t *idx_offsets, int64_t *idx,
+                                                          const int64_t *Kp, int64_t Ks, int64_t dense_K,
+                                                          int64_t *idx_offsets, int64_t *idx,
                                                           int keys_in_smem, int32_t *st) {
     extern __shared__ uint32_t keys[];
     __shared__ uint32_t hist[256];
@@ -117,7 +141,18 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float *__restric
         int64_t a, n;
         row_bounds(offsets, r, T, a, n);
         const int64_t K = row_K(Kp, Ks, r, nullptr);
-        int64_t *out = idx + idx_offsets[r];
+        int64_t obase;
+        if (dense_K > 0) {
+            const int64_t per = T < dense_K ? T : dense_K;
+            obase = r * per;
+            if (tid == 0) {
+                idx_offsets[r] = obase;
+                if (r == rows - 1) idx_offsets[rows] = rows * per;
+            }
+        } else {
+            obase = idx_offsets[r];
+        }
+        int64_t *out = idx + obase;
         if (n <= 0) continue;
         if (K >= n) {
             for (int64_t t = tid; t < n; t += kThreads) out[t] = t;
@@ -146,9 +181,11 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float *__restric
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int b = tid; b < 256; b += kThreads) hist[b] = 0;
             __syncthreads();
-            for (int64_t j = tid; j < m; j += kThreads) {
-                const uint32_t k = in_smem ? keys[j] : key_of(row[j]);
-                if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            for (int64_t base = 0; base < m; base += kThreads) {   // uniform trip count: whole warps
+                const int64_t j = base + tid;
+                uint32_t k = 0;
+                if (j < m) k = in_smem ? keys[j] : key_of(row[j]);
+                hist_add(hist, j < m && (k & mask) == prefix, (k >> shift) & 255u);
             }
             __syncthreads();
             if (tid < 32) {
@@ -184,20 +221,43 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float *__restric
             rem = s_rem;
             __syncthreads();
         }
-        // ordered compaction: key > v, or key == v among the first `rem` equal keys
+        // ordered compaction: key > v, or key == v among the first `rem` equal keys.  Each thread
+        // takes kPerThread consecutive keys of a tile; two block scans per tile place its output.
         const uint32_t v = prefix;
         int64_t carry_eq = 0, carry_sel = 0;
-        for (int64_t base = 0; base < m; base += kThreads) {
-            const int64_t j = base + tid;
-            uint32_t k = 0;
-            if (j < m) k = in_smem ? keys[j] : key_of(row[j]);
-            const int eq = (j < m && k == v) ? 1 : 0;
+        for (int64_t base = 0; base < m; base += kTile) {
+            const int64_t j0 = base + (int64_t)tid * kPerThread;
+            uint32_t kk[kPerThread];
+            int n_eq = 0, n_gt = 0;
+#pragma unroll
+            for (int q = 0; q < kPerThread; ++q) {
+                const int64_t j = j0 + q;
+                kk[q] = 0;
+                if (j < m) kk[q] = in_smem ? keys[j] : key_of(row[j]);
+                n_eq += (j < m && kk[q] == v) ? 1 : 0;
+                n_gt += (j < m && kk[q] > v) ? 1 : 0;
+            }
             int tot_eq;
-            const int eq_rank = block_excl_scan(eq, wsum, &tot_eq);
-            const int sel = (j < m && (k > v || (eq && carry_eq + eq_rank < rem))) ? 1 : 0;
+            const int eq_base = block_excl_scan(n_eq, wsum, &tot_eq);
+            // equal keys of this thread that are still within the first `rem` of the row
+            const int64_t left = rem - (carry_eq + eq_base);
+            const int take_eq = left <= 0 ? 0 : (left >= n_eq ? n_eq : (int)left);
             int tot_sel;
-            const int pos = block_excl_scan(sel, wsum, &tot_sel);
-            if (sel) out[1 + carry_sel + pos] = j + 1;
+            const int sel_base = block_excl_scan(n_gt + take_eq, wsum, &tot_sel);
+            int64_t o = 1 + carry_sel + sel_base;
+            int eq_seen = 0;
+#pragma unroll
+            for (int q = 0; q < kPerThread; ++q) {
+                const int64_t j = j0 + q;
+                if (j < m) {
+                    const bool eq = kk[q] == v;
+                    if (kk[q] > v || (eq && eq_seen < take_eq)) {
+                        if (dcheck(o <= need, st)) out[o] = j + 1;     // slots 1 .. K-1 of the row
+                        ++o;
+                    }
+                    eq_seen += eq ? 1 : 0;
+                }
+            }
             carry_eq += tot_eq;
             carry_sel += tot_sel;
         }
@@ -220,6 +280,7 @@ extern "C" dbc_status chunk_topk_select(const float *dR, const int64_t *offsets,
                                         int64_t K_scalar, int64_t *idx, int64_t *idx_offsets,
                                         void *ws, size_t ws_bytes, int32_t *dev_status,
                                         dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_topk_select");
     (void)ws; (void)ws_bytes;
     if (rows < 0 || T < 0 || N < 0) return DBC_ERR_INVALID_ARG;
     if (!K_per_row && K_scalar < 1) return DBC_ERR_INVALID_ARG;
@@ -227,16 +288,19 @@ extern "C" dbc_status chunk_topk_select(const float *dR, const int64_t *offsets,
     if (!idx_offsets) return DBC_ERR_INVALID_ARG;
     if (rows > 0 && N > 0 && (!dR || !idx)) return DBC_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    tk::offsets_kernel<<<1, 1024, 0, s>>>(offsets, rows, T, K_per_row, K_scalar, idx_offsets,
-                                          dev_status);
-    count_launches(1);
+    // dense rows with one K: the select kernel writes the offsets itself (r * min(K, T))
+    const int64_t dense_K = (!offsets && !K_per_row) ? K_scalar : 0;
+    if (!dense_K || rows == 0 || N == 0) {
+        tk::offsets_kernel<<<1, 1024, 0, s>>>(offsets, rows, T, K_per_row, K_scalar, idx_offsets, dev_status);
+        count_launches(1);
+    }
     if (rows == 0 || N == 0) return launch_status();
     const int64_t m = T > 1 ? T - 1 : 1;
     const int keys = (int)std::min<int64_t>(m, tk::kSmemKeys);
     const size_t smem = (size_t)keys * sizeof(uint32_t);
     cudaFuncSetAttribute(tk::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int grid = (int)std::min<int64_t>(rows, 65535);
-    tk::select_kernel<<<grid, tk::kThreads, smem, s>>>(dR, offsets, rows, T, K_per_row, K_scalar,
+    tk::select_kernel<<<grid, tk::kThreads, smem, s>>>(dR, offsets, rows, T, K_per_row, K_scalar, dense_K,
                                                        idx_offsets, idx, keys, dev_status);
     count_launches(1);
     return launch_status();
