@@ -13,7 +13,9 @@ report):
 * :func:`chunk_topk_select`  BOS + the K-1 largest dR (t >= 1), in time order;
 * :func:`chunk_gather`       z_k = h_{s_k} (optionally times W_proj);
 * :func:`chunk_upsample`     S_t = h_t + g_{c(t)} W_{b(t)};
-* :func:`hnet_route`         cosine router p_t, boundaries, chunk list, EMA.
+* :func:`hnet_route`         cosine router p_t, boundaries, chunk list, EMA;
+* :func:`canon_conv1d`       the encoder's Canon layer (causal depthwise conv, k = 4),
+  :func:`chunk_coding_rate_canon` the Canon layer and the coding rate in one call.
 """
 from __future__ import annotations
 
@@ -27,7 +29,7 @@ __all__ = [
     "chunk_coding_rate_stream_workspace", "chunk_topk_select",
     "chunk_gather", "chunk_upsample", "chunk_upsample_workspace", "chunk_upsample_noalloc",
     "chunk_upsample_backward", "chunk_upsample_backward_workspace", "chunk_gather_backward",
-    "hnet_route", "hnet_route_workspace", "chunk",
+    "hnet_route", "hnet_route_workspace", "chunk", "canon_conv1d", "chunk_coding_rate_canon",
     "DBC_F32", "DBC_BF16", "BIN_OFFSET", "BIN_FRACTION", "BIN_ABSOLUTE",
     "ERR_NONFINITE", "ERR_TIMEOUT", "ERR_BOUNDS",
 ]
@@ -37,7 +39,8 @@ BIN_OFFSET, BIN_FRACTION, BIN_ABSOLUTE = 0, 1, 2
 ERR_NONFINITE, ERR_TIMEOUT, ERR_BOUNDS = 4, 5, 6
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_HERE, "libdbc.so")
+# DBC_LIBRARY=debug selects the debug build (device-side invariant checks, see build.py)
+lib_path = os.path.join(_HERE, "libdbc_debug.so" if os.environ.get("DBC_LIBRARY") == "debug" else "libdbc.so")
 _lib = None
 
 _i64, _sz, _vp, _int, _f32 = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -64,6 +67,9 @@ _SIGS = {
                                        _int, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "chunk_gather_backward": (_int, [_vp, _i64, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _int, _vp, _vp]),
     "hnet_route_workspace": (_sz, [_i64, _i64, _i64]),
+    "canon_conv1d": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp]),
+    "chunk_coding_rate_canon": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _int, _vp, _f32, _vp, _vp, _sz,
+                                       _vp, _vp]),
     "hnet_route": (_int, [_vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _f32, _int, _vp, _vp, _vp, _vp,
                           _vp, _vp, _sz, _vp, _vp]),
 }
@@ -387,3 +393,39 @@ def chunk(H, K: int, eps2: float, *, stream=None):
     Z = chunk_gather(H, idx, io, rows=rows, T=T, stream=stream)
     k = min(K, T)
     return dR.view(rows, T), idx.view(rows, k), Z.view(rows, k, d)
+
+
+def canon_conv1d(H, w, bias=None, *, offsets=None, T: Optional[int] = None, residual: bool = False, out=None,
+                 dev_status=None, stream=None):
+    """Canon layer: out_t = bf16(bias (+ h_t) + sum_j w[:, j] h_{t-j}), per row, causal (bf16 in/out)."""
+    torch = _torch()
+    _require_cuda(H, w, bias, offsets)
+    rows, T, N, d, H2 = _layout(H, offsets, T)
+    H2 = H2.contiguous()
+    if out is None:
+        out = torch.empty(N, d, dtype=torch.bfloat16, device=H.device)
+    rc = lib().canon_conv1d(_ptr(H2), _ptr(offsets), rows, T, N, d, _ptr(w.contiguous()),
+                            _ptr(bias.contiguous() if bias is not None else None), int(bool(residual)), _ptr(out),
+                            _ptr(dev_status), _stream(stream))
+    _check("canon_conv1d", rc)
+    return out
+
+
+def chunk_coding_rate_canon(H, w, eps2: float, bias=None, *, offsets=None, T: Optional[int] = None,
+                            residual: bool = False, Hc=None, dR=None, workspace=None, dev_status=None, stream=None):
+    """(Hc, dR): the Canon layer's output and its marginal coding rate, in one call."""
+    torch = _torch()
+    _require_cuda(H, w, bias, offsets)
+    rows, T, N, d, H2 = _layout(H, offsets, T)
+    H2 = H2.contiguous()
+    if Hc is None:
+        Hc = torch.empty(N, d, dtype=torch.bfloat16, device=H.device)
+    if dR is None:
+        dR = torch.empty(N, dtype=torch.float32, device=H.device)
+    ws = _workspace(chunk_coding_rate_workspace(rows, T, N, d), H.device, workspace)
+    rc = lib().chunk_coding_rate_canon(_ptr(H2), _ptr(offsets), rows, T, N, d, _ptr(w.contiguous()),
+                                       _ptr(bias.contiguous() if bias is not None else None), int(bool(residual)),
+                                       _ptr(Hc), float(eps2), _ptr(dR), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                       _stream(stream))
+    _check("chunk_coding_rate_canon", rc)
+    return Hc, dR

@@ -273,7 +273,10 @@ DBC_API dbc_status chunk_gather_backward(const float *dZ, int64_t d, const int64
  * (use chunk_upsample with a caller workspace instead).
  * The first call made with a given device current looks up the array's device
  * address (cudaGetSymbolAddress) and caches it; make that first call before
- * any stream capture.  All calls share the one array, which keeps the last
+ * any stream capture.  The cached address belongs to the device's context:
+ * after cudaDeviceReset (or any other teardown of that context) it is stale,
+ * so do not call this entry point on that device again in the same process.
+ * All calls share the one array, which keeps the last
  * call's contents (the call clears what must start at zero): calls that can
  * overlap on the GPU -- concurrent streams or host threads on one device --
  * race on it and must be serialised by the caller.
@@ -284,6 +287,42 @@ DBC_API dbc_status chunk_upsample_noalloc(const void *G, int64_t d_g, const void
                                           const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
                                           const void *W_bin, int nbins, int mode, float *S,
                                           int32_t *dev_status, dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * canon_conv1d -- the Canon layer of the local encoder: a causal depthwise
+ * convolution with kernel 4 over each row.
+ *
+ * ByteFlow (notes "Key design 1": every local-encoder layer adds a Canon
+ * layer, a causal 1-D convolution of kernel 4; summary "Method steps", stage
+ * 1: SWA + Canon(causal_conv1d, k = 4) + SwiGLU, whose output h feeds the
+ * chunker).  Reading used (per channel f, positions before a row's start = 0):
+ *   out_t[f] = bf16( bias[f] (+ h_t[f] when residual) + sum_{j=0..3} w[f*4+j] h_{t-j}[f] )
+ * accumulated in fp32 in that order (bias, residual, taps 0..3), one
+ * round-to-nearest-even to bf16.
+ *
+ * H        bf16 [N, d]; offsets NULL (dense rows of length T) or int64 [rows+1].
+ * w        bf16 [d, 4] taps (w[f*4 + j] multiplies h_{t-j}); bias bf16 [d] or NULL.
+ * out      bf16 [N, d], must not overlap H.  H and out 16-byte aligned.
+ * Supported: d a multiple of 8 up to 4096.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA; device flag BOUNDS (malformed offsets).
+ * ------------------------------------------------------------------------- */
+DBC_API dbc_status canon_conv1d(const void *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N,
+                                int64_t d, const void *w, const void *bias, int residual, void *out,
+                                int32_t *dev_status, dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * chunk_coding_rate_canon -- canon_conv1d followed by chunk_coding_rate on its
+ * output, in one call (the chunker's input is the Canon layer's output).
+ *
+ * Writes Hc = canon_conv1d(H, ...) (bf16 [N, d], kept for the gather and the
+ * upsampling's residual) and dR = the coding rate of Hc.  d in {64, 128, 256,
+ * 512}; ws of chunk_coding_rate_workspace(rows, T, N, d) bytes.
+ * Errors: as canon_conv1d and chunk_coding_rate.
+ * ------------------------------------------------------------------------- */
+DBC_API dbc_status chunk_coding_rate_canon(const void *H, const int64_t *offsets, int64_t rows, int64_t T,
+                                           int64_t N, int64_t d, const void *w, const void *bias, int residual,
+                                           void *Hc, float eps2, float *dR, void *ws, size_t ws_bytes,
+                                           int32_t *dev_status, dbc_stream_t stream);
 
 /* -------------------------------------------------------------------------
  * hnet_route -- cosine-similarity boundary router with EMA smoothing.
