@@ -1,6 +1,11 @@
 """Build libdbc.so (all kernels + the C ABI) for sm_100a with nvcc, in-tree.
 
-Usage: python -m dynamic_byte_chunking_b200.build [--force] [--verbose]
+``--debug`` builds libdbc_debug.so instead: the same library compiled with
+-DDBC_DEBUG, whose kernels check internal index invariants on the device and
+flag DBC_ERR_BOUNDS (never trap).  The binding loads it when the environment
+variable DBC_LIBRARY is set to ``debug``.
+
+Usage: python -m dynamic_byte_chunking_b200.build [--force] [--verbose] [--debug]
 """
 from __future__ import annotations
 
@@ -14,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdbc.so")
+LIB_DEBUG = os.path.join(PKG, "libdbc_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -29,24 +35,26 @@ def _deps():
     return _sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "dbc.h")]
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(debug: bool = False) -> bool:
+    lib = LIB_DEBUG if debug else LIB
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -> str:
-    """Compile every csrc/*.cu to an object, then link libdbc.so."""
-    if not force and not needs_build():
-        return LIB
-    objdir = os.path.join(PKG, "_build")
+def build(force: bool = False, verbose: bool = False, jobs: int | None = None, debug: bool = False) -> str:
+    """Compile every csrc/*.cu to an object, then link libdbc.so (libdbc_debug.so with debug=True)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not needs_build(debug):
+        return lib
+    objdir = os.path.join(PKG, "_build_debug" if debug else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, procs = [], []
     for src in _sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
-        cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [NVCC, *ARCH, *FLAGS, *(["-DDBC_DEBUG"] if debug else []), "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
@@ -60,13 +68,12 @@ def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(os.path.basename(f) for f in failed))
-    tmp = LIB + f".{os.getpid()}.tmp"
+    tmp = lib + f".{os.getpid()}.tmp"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt",
                            "-lpthread"])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

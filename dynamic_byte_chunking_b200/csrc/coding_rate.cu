@@ -638,6 +638,7 @@ extern "C" dbc_status chunk_coding_rate(const void *H, int dtype, const int64_t 
                                         int64_t rows, int64_t T, int64_t N, int64_t d,
                                         float eps2, float *dR, void *ws, size_t ws_bytes,
                                         int32_t *dev_status, dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_coding_rate");
     if (rows < 0 || T < 0 || N < 0 || !(eps2 > 0.f) || !isfinite(eps2)) return DBC_ERR_INVALID_ARG;
     if (dtype != DBC_F32 && dtype != DBC_BF16) return DBC_ERR_UNSUPPORTED;
     if (d != 64 && d != 128 && d != 256 && d != 512) return DBC_ERR_UNSUPPORTED;
@@ -687,6 +688,7 @@ extern "C" size_t chunk_coding_rate_stream_workspace(int64_t streams, int64_t n,
 extern "C" dbc_status chunk_coding_rate_stream(const void *H, int dtype, int64_t streams, int64_t n, int64_t d,
                                                int64_t t0, float eps2, double *state, float *dR, void *ws,
                                                size_t ws_bytes, int32_t *dev_status, dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_coding_rate_stream");
     if (streams < 0 || n < 0 || t0 < 0 || !(eps2 > 0.f) || !isfinite(eps2)) return DBC_ERR_INVALID_ARG;
     if (dtype != DBC_BF16 || d != 256) return DBC_ERR_UNSUPPORTED;
     if (streams == 0 || n == 0) return DBC_OK;

@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <algorithm>
@@ -42,6 +43,23 @@ __device__ __forceinline__ void flag(int32_t *st, int code) {
     if (st) atomicOr(st, 1 << code);
 }
 
+// Internal invariants checked on the device in the debug build (compiled with
+// -DDBC_DEBUG, libdbc_debug.so): a violated invariant flags DBC_ERR_BOUNDS and
+// the caller skips the access instead of trapping.  The release build
+// compiles the check away (it always passes).
+#ifdef DBC_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool dcheck(bool cond, int32_t *st) {
+    if (kDebugChecks && !cond) {
+        flag(st, DBC_ERR_BOUNDS);
+        return false;
+    }
+    return true;
+}
+
 __device__ __forceinline__ float ld_f(const float *p) { return *p; }
 __device__ __forceinline__ float ld_f(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
@@ -66,6 +84,16 @@ __device__ __forceinline__ int64_t find_row(const int64_t *offs, int64_t rows, i
     }
     return lo;
 }
+
+// Names one C-ABI call in profiler timelines (an NVTX range; header-only, and
+// without an attached tool each push/pop is a call through a null hook).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+#define DBC_NVTX_RANGE(name) ::dbc::NvtxRange dbc_nvtx_range_(name)
 
 // Number of kernels the library has launched (all entry points, all threads).
 void count_launches(int n);

@@ -379,6 +379,7 @@ extern "C" dbc_status hnet_route(const void *H, const int64_t *offsets, int64_t 
                                  int do_ema, float *p, uint8_t *boundary, int64_t *chunk_idx,
                                  int64_t *chunk_offsets, float *z_smooth, void *ws, size_t ws_bytes,
                                  int32_t *dev_status, dbc_stream_t stream) {
+    DBC_NVTX_RANGE("hnet_route");
     if (rows < 0 || T < 0 || N < 0 || !isfinite(threshold)) return DBC_ERR_INVALID_ARG;
     if (d != 64 && d != 128 && d != 256 && d != 512) return DBC_ERR_UNSUPPORTED;
     if (!offsets && N != rows * T) return DBC_ERR_INVALID_ARG;

@@ -118,7 +118,7 @@ template <class IN>
 __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16 *__restrict__ G, int64_t dg,
                                                              const IN *__restrict__ H, int64_t dl,
                                                              const __nv_bfloat16 *__restrict__ W, int nbins,
-                                                             Layout L, float *__restrict__ S, int32_t *st) {
+                                                             Layout L, float *__restrict__ S, int64_t N, int32_t *st) {
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[BinTC::NS];
     __shared__ uint32_t tmem_base;
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16
 #pragma unroll 1
         for (int rr = warp; rr < 128; rr += 8) {
             const int p = pos[rr];
-            if (p < 0) continue;
+            if (p < 0 || !dcheck(p < N, st)) continue;
             for (int c8 = lane; c8 < nvec; c8 += 32) {
                 const float *t = tile + rr * LDT + c8 * 8;
                 const float4 a0 = *reinterpret_cast<const float4 *>(t);
@@ -275,13 +275,13 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
                              (int)BinTC::smem<__nv_bfloat16>());
         bin_gemm_tc_kernel<__nv_bfloat16><<<g, 256, BinTC::smem<__nv_bfloat16>(), s>>>(
             static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
+            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, N, dev_status);
     } else {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)BinTC::smem<float>());
         bin_gemm_tc_kernel<float><<<g, 256, BinTC::smem<float>(), s>>>(
             static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, dev_status);
+            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, N, dev_status);
     }
     count_launches(4);
     return launch_status();
@@ -303,6 +303,7 @@ extern "C" dbc_status chunk_upsample(const void *G, int64_t d_g, const void *H, 
                                      const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
                                      const void *W_bin, int nbins, int mode, float *S, void *ws,
                                      size_t ws_bytes, int32_t *dev_status, dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_upsample");
     if (rows < 0 || T < 0 || N < 0 || d_g <= 0 || d_l <= 0) return DBC_ERR_INVALID_ARG;
     if (nbins < 1 || nbins > up::kMaxBins) return DBC_ERR_INVALID_ARG;
     if (mode < DBC_BIN_IN_CHUNK_OFFSET || mode > DBC_BIN_ABSOLUTE) return DBC_ERR_INVALID_ARG;
@@ -367,6 +368,7 @@ extern "C" dbc_status chunk_upsample_noalloc(const void *G, int64_t d_g, const v
                                              const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
                                              const void *W_bin, int nbins, int mode, float *S,
                                              int32_t *dev_status, dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_upsample_noalloc");
     if (rows < 0 || T < 0 || N < 0 || d_g <= 0 || d_l <= 0) return DBC_ERR_INVALID_ARG;
     if (nbins < 1 || nbins > up::kMaxBins) return DBC_ERR_INVALID_ARG;
     if (mode < DBC_BIN_IN_CHUNK_OFFSET || mode > DBC_BIN_ABSOLUTE) return DBC_ERR_INVALID_ARG;

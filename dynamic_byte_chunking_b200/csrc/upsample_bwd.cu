@@ -651,6 +651,7 @@ extern "C" dbc_status chunk_upsample_backward(const float *dS, const void *G, in
                                               const void *W_bin, int nbins, int mode, float *dG, float *dW,
                                               float *dH, void *ws, size_t ws_bytes, int32_t *dev_status,
                                               dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_upsample_backward");
     if (rows < 0 || T < 0 || N < 0 || total_K < 0 || d_g <= 0 || d_l <= 0) return DBC_ERR_INVALID_ARG;
     if (nbins < 1 || nbins > ub::kMaxBins) return DBC_ERR_INVALID_ARG;
     if (mode < DBC_BIN_IN_CHUNK_OFFSET || mode > DBC_BIN_ABSOLUTE) return DBC_ERR_INVALID_ARG;
@@ -704,6 +705,7 @@ extern "C" dbc_status chunk_gather_backward(const float *dZ, int64_t d, const in
                                             const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
                                             int64_t total_K, float *dH, int accumulate, int32_t *dev_status,
                                             dbc_stream_t stream) {
+    DBC_NVTX_RANGE("chunk_gather_backward");
     if (rows < 0 || T < 0 || total_K < 0 || d <= 0) return DBC_ERR_INVALID_ARG;
     if (d % 4) return DBC_ERR_UNSUPPORTED;
     if (total_K == 0 || rows == 0) return DBC_OK;

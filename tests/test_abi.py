@@ -37,6 +37,17 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n), n
 
 
+def test_debug_library_exports_every_symbol():
+    """The debug build (device-side invariant checks, -DDBC_DEBUG) links and exports the same ABI."""
+    from dynamic_byte_chunking_b200 import build
+    path = build.build(debug=True)
+    D = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(D, n), n
+    D.dbc_status_string.restype = ctypes.c_char_p
+    assert D.dbc_status_string(6) == b"DBC_ERR_BOUNDS"
+
+
 def test_status_strings_and_version(L):
     import dynamic_byte_chunking_b200 as dbc
     assert dbc.status_string(0) == "DBC_OK"
