@@ -10,7 +10,8 @@ Metric: sequence bytes per second (byte positions of the batch / step time).
 Timing: W untimed warm-up steps, then exactly K steps, each preceded (outside
 its timed interval) by a 256 MB write that flushes the 126 MB L2; CUDA events
 on the launching stream; barrier + synchronize around the timed loop; max over
-ranks.  Under torchrun each rank runs its own batch (weak scaling, no
+ranks.  Under torchrun one global batch of 8 rows per rank is drawn and its
+rows are split over the ranks by the library's row partition (weak scaling, no
 collective on the data path).
 
 ``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
@@ -355,7 +356,21 @@ def run_rows(args):
             ms = _time(stream_pass, args.reps, flush, stream)
             emit("NEXT-2 streaming coding rate (blocks of 256)", fam, ms, positions_per_s=N / (ms * 1e-3),
                  blocks=len(blocks), us_per_block=ms * 1e3 / len(blocks), tflops=fl / (ms * 1e-3) / 1e12)
-            del blocks, state, dRs, wss
+            # latency of the smallest block: one new position per stream, 64 calls in a row mid-sequence
+            t_mid = 4096
+            ones = [Hs[:, t:t + 1, :].contiguous() for t in range(t_mid, t_mid + 64)]
+            ws1 = torch.empty(max(dbc.chunk_coding_rate_stream_workspace(rows, 1, t, d) for t in range(t_mid, t_mid + 64)),
+                              dtype=torch.uint8, device=dev)
+            dR1 = torch.empty(rows, dtype=torch.float32, device=dev)
+
+            def byte_steps():
+                for j, b in enumerate(ones):
+                    dbc.chunk_coding_rate_stream(b, w.eps2, state, t_mid + j, dR=dR1, workspace=ws1)
+
+            ms1 = _time(byte_steps, args.reps, flush, stream)
+            emit("NEXT-2 streaming coding rate (one position per call)", fam, ms1, calls=len(ones),
+                 us_per_call=ms1 * 1e3 / len(ones), streams=rows)
+            del blocks, state, dRs, wss, ones, ws1, dR1
         if w.dtype == "bf16":
             # NEXT-4: the encoder's Canon layer (causal depthwise conv, k = 4) alone and chained with the chunker
             gen = np.random.default_rng(11)
@@ -475,10 +490,15 @@ def main():
         pg = dist
     stream = torch.cuda.current_stream()
 
-    w = workloads.make("byteflow", seed=1 + rank)
-    rows, T, d, K = w.rows, w.T, w.d, int(w.K[0])
-    N = w.N
-    H_host = torch.from_numpy(w.H_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    # one global batch of 8 rows per rank (weak scaling), its rows split over the ranks by the
+    # library's row partition (contiguous blocks for a dense batch); no collective on the data path
+    from dynamic_byte_chunking_b200 import sharding
+    w = workloads.make("byteflow", seed=1, rows=8 * world)
+    mine = sharding.partition_rows(w.lengths, world)[rank]
+    H_bits, _ = sharding.shard_rows_host(w.H_bits, w.offsets, mine)
+    rows, T, d, K = len(mine), w.T, w.d, int(w.K[0])
+    N = rows * T
+    H_host = torch.from_numpy(np.ascontiguousarray(H_bits).view(np.int16)).view(torch.bfloat16).pin_memory()
     H = H_host.to(dev).view(rows, T, d)
     Wb = torch.from_numpy(w.W_bin.view(np.int16)).view(torch.bfloat16).to(dev)
     nb = Wb.shape[0]
@@ -654,7 +674,8 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": WORKLOAD, "rows_per_gpu": rows, "T": T, "d": d, "K": K, "nbins": nb,
-                           "global_batch": rows * world, "parallelism": f"dp{world} (independent rows)",
+                           "global_batch": 8 * world,
+                           "parallelism": f"dp{world}: rows of one global batch split by sharding.partition_rows",
                            "l2": "flushed by a 256 MB write before every timed step",
                            "step": " -> ".join(stages)},
                 "stage_ms": {s: float(a) for s, a in zip(stages, avg)},

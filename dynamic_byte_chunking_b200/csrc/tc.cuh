@@ -36,6 +36,12 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
     return d;
 }
 
+// The same descriptor moved by `bytes` (a multiple of 16): only the start
+// address field changes, and it does not carry out of its 14 bits for shared
+// memory addresses below 256 KB.  Lets an MMA loop build one descriptor per
+// tile and add constant offsets instead of rebuilding it.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
 // kind::f16 instruction descriptor: bf16 x bf16 -> fp32, M x N; negate_a
 // turns the MMA into D -= A B^T.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major,

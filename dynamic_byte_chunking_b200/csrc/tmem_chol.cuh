@@ -19,7 +19,8 @@
 //  * FACTOR (segment start state M_s = I + P_s = L L^T): the upper triangle,
 //    which starts at zero, carries B = L^{-T} along (row i of the identity
 //    solved against the factor, B_ii = 1 / L_ii), so one sweep yields it;
-//    the panels of B are stored as three bf16 pieces.  Since
+//    each solved panel is written back to TMEM and B leaves for global memory
+//    once, as three bf16 pieces, after the last panel.  Since
 //    M_s^{-1} = B B^T, the whitened rows Y = sqrt(c) X_s B give the segment's
 //    problem c X_s M_s^{-1} X_s^T = Y Y^T.
 //  * INSEG (one segment): G' = Y Y^T (Y in three pieces, six piece
@@ -51,14 +52,19 @@ struct TmemChol {
 __device__ __forceinline__ constexpr int pair_a(int i) { return i == 2 ? 1 : (i == 4 ? 2 : (i == 5 ? 1 : 0)); }
 __device__ __forceinline__ constexpr int pair_b(int i) { return i == 1 ? 1 : (i == 3 ? 2 : (i == 5 ? 1 : 0)); }
 
-__device__ __forceinline__ void split3v(float v, uint16_t &h, uint16_t &m, uint16_t &l) {
-    const __nv_bfloat16 bh = __float2bfloat16_rn(v);
-    const float r1 = v - __bfloat162float(bh);
-    const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 bl = __float2bfloat16_rn(r1 - __bfloat162float(bm));
-    h = __bfloat16_as_ushort(bh);
-    m = __bfloat16_as_ushort(bm);
-    l = __bfloat16_as_ushort(bl);
+// Two values split at once into three packed bf16x2 pieces (hi, mid, lo): the
+// round-to-nearest-even pieces whose sum carries the fp32 value, one paired
+// conversion each.
+__device__ __forceinline__ void split3x2(float a, float b, uint32_t &h, uint32_t &m, uint32_t &l) {
+    const __nv_bfloat162 bh = __floats2bfloat162_rn(a, b);
+    const float2 fh = __bfloat1622float2(bh);
+    const float ra = a - fh.x, rb = b - fh.y;
+    const __nv_bfloat162 bm = __floats2bfloat162_rn(ra, rb);
+    const float2 fm = __bfloat1622float2(bm);
+    const __nv_bfloat162 bl = __floats2bfloat162_rn(ra - fm.x, rb - fm.y);
+    h = *reinterpret_cast<const uint32_t *>(&bh);
+    m = *reinterpret_cast<const uint32_t *>(&bm);
+    l = *reinterpret_cast<const uint32_t *>(&bl);
 }
 
 // Stages 64 values of one row as three K-major pieces (row `row` of each
@@ -70,14 +76,7 @@ __device__ __forceinline__ void stage_row(uint32_t region, int row, const float 
     for (int k8 = 0; k8 < 8; ++k8) {
         uint32_t hh[4], mm[4], ll[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint16_t h0, m0, l0, h1, m1, l1;
-            split3v(a[k8 * 8 + 2 * q], h0, m0, l0);
-            split3v(a[k8 * 8 + 2 * q + 1], h1, m1, l1);
-            hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-            mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
-            ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-        }
+        for (int q = 0; q < 4; ++q) split3x2(a[k8 * 8 + 2 * q], a[k8 * 8 + 2 * q + 1], hh[q], mm[q], ll[q]);
         const uint32_t off = tc::kmajor_off(row, k8 * 8);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + off), "r"(hh[0]), "r"(hh[1]),
                      "r"(hh[2]), "r"(hh[3])
@@ -96,63 +95,39 @@ __device__ __forceinline__ void stage_row(uint32_t region, int row, const float 
     }
 }
 
-// D[block b rows, columns c0 .. c0+N) (+/-)= sum of the six piece products of
-// A (rows a_row0 .. +128 of the staged tiles) and B (rows b_row0 .. +N).
-__device__ __forceinline__ void issue_split_mma(uint32_t d_tmem, uint32_t region_a, uint32_t region_b,
-                                                int a_row0, int b_row0, uint32_t idesc, bool first) {
-#pragma unroll
-    for (int pr = 0; pr < 6; ++pr) {
-        const uint32_t pa = region_a + (uint32_t)pair_a(pr) * TmemChol::PIECE + (uint32_t)a_row0 * 128;
-        const uint32_t pb = region_b + (uint32_t)pair_b(pr) * TmemChol::PIECE + (uint32_t)b_row0 * 128;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(d_tmem, tc::sdesc(pa + kk * 32, 16, 1024), tc::sdesc(pb + kk * 32, 16, 1024), idesc,
-                         (first && pr == 0 && kk == 0) ? 0u : 1u);
-    }
-}
-
-// Stages 16 values of one row as three K-major pieces (K = 16: the first two
-// 16-byte chunks of the row's 128-byte line in each 256-row tile).
-__device__ __forceinline__ void stage_row16(uint32_t region, int row, const float (&a)[16]) {
-#pragma unroll
-    for (int k8 = 0; k8 < 2; ++k8) {
-        uint32_t hh[4], mm[4], ll[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint16_t h0, m0, l0, h1, m1, l1;
-            split3v(a[k8 * 8 + 2 * q], h0, m0, l0);
-            split3v(a[k8 * 8 + 2 * q + 1], h1, m1, l1);
-            hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-            mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
-            ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-        }
-        const uint32_t off = tc::kmajor_off(row, k8 * 8);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + off), "r"(hh[0]), "r"(hh[1]),
-                     "r"(hh[2]), "r"(hh[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + TmemChol::PIECE + off), "r"(mm[0]),
-                     "r"(mm[1]), "r"(mm[2]), "r"(mm[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(region + 2 * TmemChol::PIECE + off),
-                     "r"(ll[0]), "r"(ll[1]), "r"(ll[2]), "r"(ll[3])
-                     : "memory");
-    }
-}
-
 // D[block rows, columns j1 ..) -= sum of the six piece products over K = 16:
 // A = staged rows a_row0 .. +128, B = staged rows b_row0 .. +N.
-__device__ __forceinline__ void issue_split_mma_k16(uint32_t d_tmem, uint32_t region, int a_row0, int b_row0,
+// `dreg` is the descriptor of the staging region's first byte (K-major, SBO 1024).
+__device__ __forceinline__ void issue_split_mma_k16(uint32_t d_tmem, uint64_t dreg, int a_row0, int b_row0,
                                                     uint32_t idesc) {
+    const uint64_t da = tc::sdesc_add(dreg, (uint32_t)a_row0 * 128), db = tc::sdesc_add(dreg, (uint32_t)b_row0 * 128);
 #pragma unroll
-    for (int pr = 0; pr < 6; ++pr) {
-        const uint32_t pa = region + (uint32_t)pair_a(pr) * TmemChol::PIECE + (uint32_t)a_row0 * 128;
-        const uint32_t pb = region + (uint32_t)pair_b(pr) * TmemChol::PIECE + (uint32_t)b_row0 * 128;
-        tc::mma_bf16(d_tmem, tc::sdesc(pa, 16, 1024), tc::sdesc(pb, 16, 1024), idesc, 1u);
-    }
+    for (int pr = 0; pr < 6; ++pr)
+        tc::mma_bf16(d_tmem, tc::sdesc_add(da, (uint32_t)pair_a(pr) * TmemChol::PIECE),
+                     tc::sdesc_add(db, (uint32_t)pair_b(pr) * TmemChol::PIECE), idesc, 1u);
 }
 
 // Runtime N of the negated trailing update (N = 256 - j1, a multiple of 64).
 __device__ __forceinline__ uint32_t idesc_neg(int N) { return tc::idesc_bf16(128, N, false, false, true); }
+
+// Block-wide barrier and AND-vote of the 256 threads (named barrier 1).
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool cbar_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.and.pred p, 1, 256, q;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
+// Pair pi of the in-segment Y GEMM -> (output chunk c, K chunk k), k <= c < 4.
+__device__ __forceinline__ void ypair(int pi, int &c, int &k) {
+    c = 0;
+    k = pi;
+    while (k > c) { k -= c + 1; ++c; }
+}
 
 template <bool FACTOR>
 __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
@@ -166,9 +141,14 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     __shared__ __align__(16) float s_LdT[16][16];   // factored 16 x 16 diagonal block, column-major
     __shared__ __align__(16) float s_rl[16];        // 1 / L_kk of the diagonal block
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // MMAs are issued by one thread, lane 0 of warp 7: in-order MMA semantics need a single issuer,
+    // and warp 7 is the diagonal-block warp of only the last two panels, so the issue time is spent
+    // while the other warps factor the next diagonal block
+    const bool issuer = tid == 7 * 32;
     const int blk = warp >> 2, lb = (warp & 3) * 32;
     const int row = blk * 128 + lb + lane;
     const uint32_t region = (tc::smem_u32(smraw) + 1023u) & ~1023u;
+    const uint64_t dregion = tc::sdesc(region, 16, 1024);      // K-major tiles of the region
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) tc::mbar_init(&mbar[i], 1);
@@ -178,368 +158,425 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = tmem_base;
-    const uint32_t trow = tbase + ((uint32_t)lb << 16) + (uint32_t)(blk * 256);
-    uint32_t ph0 = 0, ph1 = 0;      // mbarrier phases (uniform across threads)
-    uint32_t phs[2] = {0, 0}, phy = 0;
-    bool ok = true;
     const int nseg = *S.nseg;
+    constexpr int NPAIR = 10;
+    constexpr uint32_t idy = tc::idesc_bf16(128, 64, false, true);
+    constexpr uint32_t idg0 = tc::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idg1 = tc::idesc_bf16(128, 256, false, false);
 
-    for (int s = blockIdx.x; s < nseg && ok; s += gridDim.x) {
-        const int len = S.len[s];
-        const int64_t start = S.start[s];
-        const int n = FACTOR ? D : len;
+    {
+        // ================= thread (warp w, lane l) owns row (w/4)*128 + (w%4)*32 + l
+        const uint32_t trow = tbase + ((uint32_t)lb << 16) + (uint32_t)(blk * 256);
+        uint32_t ph0 = 0, ph1 = 0;      // mbarrier phases (uniform across the compute threads)
+        uint32_t phs[2] = {0, 0}, phy = 0;
+        bool ok = true;
+        // A timeout makes `ok` false: every later wait and MMA is skipped (commits still arrive),
+        // and the block-wide votes keep all threads on the same path to the end.
+        for (int s = blockIdx.x; s < nseg; s += gridDim.x) {
+            const int len = S.len[s];
+            const int64_t start = S.start[s];
+            const int n = FACTOR ? D : len;
 
-        // ---------------- load the matrix into TMEM
-        if (FACTOR) {
-            const float *P = Pbuf + (size_t)s * D * D;            // c-scaled prefix Gram
-            float *stg = reinterpret_cast<float *>(smraw + (region - tc::smem_u32(smraw)));
-            for (int q = 0; q < D / 64; ++q) {
-                for (int e = tid; e < D * 16; e += TmemChol::NT) {           // 256 rows x 16 float4
-                    const int r = e >> 4, c4 = e & 15;
-                    const float4 x = *reinterpret_cast<const float4 *>(P + (size_t)r * D + q * 64 + c4 * 4);
-                    float *d = stg + r * 65 + c4 * 4;
-                    d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
-                }
-                __syncthreads();
+            // ---------------- load the matrix into TMEM
+            if (FACTOR) {
+                // each thread moves its own row of the c-scaled prefix Gram into TMEM: the lower
+                // triangle (loaded straight from global memory, 8 loads in flight) and zeros right
+                // of it, where B = L^{-T} accumulates
+                const float *P = Pbuf + (size_t)s * D * D + (size_t)row * D;
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    float4 x[8];
+                    const bool any = q * 32 <= row;                      // warp-uniform
+                    if (any) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float v[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = q * 64 + j * 16 + i;
-                        v[i] = col <= row ? stg[row * 65 + j * 16 + i] : 0.f;
+                        for (int i = 0; i < 8; ++i) x[i] = *reinterpret_cast<const float4 *>(P + q * 32 + 4 * i);
                     }
-                    tc::tmem_st16(trow + (uint32_t)(q * 64 + j * 16), v);
-                }
-                __syncthreads();
-            }
-            tc::tmem_wait_st();
-        } else {
-            // G' = Y Y^T with the whitened rows Y = sqrt(c) X_s B_s formed here, 64 features at a
-            // time: Y_c = X_s B_s[:, chunk c] accumulates in the TMEM columns 128..255 (free in this
-            // mode: the first row block only uses its lower triangle), over the K chunks k <= c (B
-            // is upper triangular) with X and the three pieces of B streamed through two cp.async
-            // stages; Y_c is then split into three bf16 pieces in shared memory and G' += Y_c Y_c^T
-            // (six piece products) is issued while the next chunk's Y MMAs follow in the pipe.
-            const __nv_bfloat16 *Xs = Hx + start * D;
-            const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
-            const uint32_t yp = region;                                    // Y_c pieces, K-major
-            auto load = [&](int pi, uint32_t sa) {
-                int c = 0, k = pi;
-                while (k > c) { k -= c + 1; ++c; }                         // pair pi -> (chunk c, K chunk k)
-                for (int e = tid; e < 256 * 8; e += TmemChol::NT) {        // X: 256 positions x 64 K
-                    const int r = e >> 3, ch = e & 7;
-                    const bool in = r < len;
-                    const uint32_t xo = (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
-                    tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + k * 64 + ch * 8, in ? 16u : 0u);
-                }
-                const uint32_t sb = sa + TmemChol::YX_BYTES;
-                for (int e = tid; e < 3 * 64 * 8; e += TmemChol::NT) {     // B: 3 pieces x 64 K x 64 N
-                    const int p = e >> 9, kr = (e >> 3) & 63, n8 = e & 7;
-                    const int krow = k * 64 + kr, col = c * 64 + n8 * 8;
-                    const bool nz = krow < (col >> 4) * 16 + 16;             // stored rows of the columns' panel
-                    tc::cp_async16(sb + (uint32_t)p * 8192 + tc::mnmajor_off(n8 * 8, kr, 8192),
-                                   Bseg + (size_t)p * D * D + (size_t)(nz ? krow : 0) * D + col, nz ? 16u : 0u);
-                }
-            };
-            constexpr int NPAIR = 10;                                      // (c, k) with k <= c < 4
-            constexpr uint32_t idy = tc::idesc_bf16(128, 64, false, true);
-            constexpr uint32_t idg0 = tc::idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idg1 = tc::idesc_bf16(128, 256, false, false);
-            const float sc = sqrtf(c_rate);
-            load(0, region + TmemChol::YSTAGE0);
-            tc::cp_async_commit();
-            for (int pi = 0; pi < NPAIR; ++pi) {
-                int c = 0, k = pi;
-                while (k > c) { k -= c + 1; ++c; }
-                if (pi + 1 < NPAIR) {
-                    const int q = (pi + 1) & 1;
-                    if (pi + 1 >= 2) {                                      // stage q was read by pair pi - 1
-                        ok &= tc::mbar_wait(&mbar[3 + q], phs[q], st);
-                        phs[q] ^= 1;
-                    }
-                    load(pi + 1, region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE);
-                }
-                tc::cp_async_commit();
-                tc::cp_async_wait<1>();
-                tc::fence_async_smem();
-                __syncthreads();
-                const uint32_t sa = region + TmemChol::YSTAGE0 + (uint32_t)(pi & 1) * TmemChol::YSTAGE;
-                if (tid == 0) {
-                    tc::fence_after_sync();
-                    const uint32_t sb = sa + TmemChol::YX_BYTES;
 #pragma unroll
-                    for (int b = 0; b < 2; ++b)
+                    for (int j = 0; j < 2; ++j) {
+                        float v[16];
 #pragma unroll
-                        for (int p = 0; p < 3; ++p)
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc::mma_bf16(tbase + (uint32_t)(128 + b * 64),
-                                             tc::sdesc(sa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
-                                             tc::sdesc(sb + (uint32_t)p * 8192 + kk * 2048, 8192, 1024), idy,
-                                             (k > 0 || p > 0 || kk > 0) ? 1u : 0u);
-                    tc::mma_commit(&mbar[3 + (pi & 1)]);
-                    if (k == c) tc::mma_commit(&mbar[5]);
-                }
-                if (k == c) {
-                    // Y_c complete (and with it every earlier MMA, so the pieces buffer is free)
-                    ok &= tc::mbar_wait(&mbar[5], phy, st);
-                    phy ^= 1;
-                    tc::fence_after_sync();
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (ok) {
-                        float a64[64];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float v16[16];
-                            tc::tmem_ld16(tbase + ((uint32_t)lb << 16) + (uint32_t)(128 + blk * 64 + q * 16), v16);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) a64[q * 16 + i] = sc * v16[i];
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = q * 32 + j * 16 + i;
+                            const float4 &f = x[(j * 16 + i) >> 2];
+                            const float e = ((i & 3) == 0) ? f.x : ((i & 3) == 1) ? f.y : ((i & 3) == 2) ? f.z : f.w;
+                            v[i] = (any && col <= row) ? e : 0.f;
                         }
-                        stage_row(yp, row, a64, nullptr, 0);
+                        tc::tmem_st16(trow + (uint32_t)(q * 32 + j * 16), v);
                     }
+                }
+                tc::tmem_wait_st();
+            } else {
+                // G' = Y Y^T with the whitened rows Y = sqrt(c) X_s B_s formed here, 64 features at
+                // a time: Y_c = X_s B_s[:, chunk c] accumulates in the TMEM columns 128..255 (free in
+                // this mode: the first row block only uses its lower triangle), over the K chunks
+                // k <= c (B is upper triangular) with X and the three pieces of B streamed through
+                // two cp.async stages; Y_c is then split into three bf16 pieces in shared memory and
+                // G' += Y_c Y_c^T (six piece products) is issued while the next chunk's operands load.
+                const __nv_bfloat16 *Xs = Hx + start * D;
+                const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
+                auto load = [&](int pi, uint32_t sa) {
+                    int c, k;
+                    ypair(pi, c, k);
+                    for (int e = tid; e < 256 * 8; e += 256) {              // X: 256 positions x 64 K
+                        const int r = e >> 3, ch = e & 7;
+                        const bool in = r < len;
+                        const uint32_t xo =
+                            (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
+                        tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + k * 64 + ch * 8, in ? 16u : 0u);
+                    }
+                    const uint32_t sb = sa + TmemChol::YX_BYTES;
+                    for (int e = tid; e < 3 * 64 * 8; e += 256) {           // B: 3 pieces x 64 K x 64 N
+                        const int p = e >> 9, kr = (e >> 3) & 63, n8 = e & 7;
+                        const int krow = k * 64 + kr, col = c * 64 + n8 * 8;
+                        const bool nz = krow < (col >> 4) * 16 + 16;         // stored rows of the columns' panel
+                        tc::cp_async16(sb + (uint32_t)p * 8192 + tc::mnmajor_off(n8 * 8, kr, 8192),
+                                       Bseg + (size_t)p * D * D + (size_t)(nz ? krow : 0) * D + col, nz ? 16u : 0u);
+                    }
+                };
+                const float sc = sqrtf(c_rate);
+                load(0, region + TmemChol::YSTAGE0);
+                tc::cp_async_commit();
+                for (int pi = 0; pi < NPAIR; ++pi) {
+                    int c, k;
+                    ypair(pi, c, k);
+                    if (pi + 1 < NPAIR) {
+                        const int q = (pi + 1) & 1;
+                        if (pi + 1 >= 2) {                                   // stage q was read by pair pi - 1
+                            if (ok) ok = tc::mbar_wait(&mbar[3 + q], phs[q], st);
+                            phs[q] ^= 1;
+                        }
+                        load(pi + 1, region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE);
+                    }
+                    tc::cp_async_commit();
+                    tc::cp_async_wait<1>();
                     tc::fence_async_smem();
-                    tc::fence_before_sync();
-                    ok = __syncthreads_and(ok) != 0;
-                    if (!ok) break;
-                    if (tid == 0) {
-                        tc::fence_after_sync();
-#pragma unroll
-                        for (int pr = 0; pr < 6; ++pr) {
-                            const uint32_t pa = yp + (uint32_t)pair_a(pr) * TmemChol::PIECE;
-                            const uint32_t pb = yp + (uint32_t)pair_b(pr) * TmemChol::PIECE;
+                    ok = cbar_and(ok);                                       // stage pi complete everywhere
+                    if (issuer) {
+                        if (ok) {
+                            tc::fence_after_sync();
+                            const uint32_t sa = region + TmemChol::YSTAGE0 + (uint32_t)(pi & 1) * TmemChol::YSTAGE;
+                            const uint64_t dxa = tc::sdesc(sa, 16, 1024);                        // X, K-major
+                            const uint64_t dbb = tc::sdesc(sa + TmemChol::YX_BYTES, 8192, 1024);  // B, MN-major
 #pragma unroll
                             for (int b = 0; b < 2; ++b)
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    tc::mma_bf16(tbase + (uint32_t)(b * 256),
-                                                 tc::sdesc(pa + (uint32_t)b * 128 * 128 + kk * 32, 16, 1024),
-                                                 tc::sdesc(pb + kk * 32, 16, 1024), b == 0 ? idg0 : idg1,
-                                                 (c > 0 || pr > 0 || kk > 0) ? 1u : 0u);
+                                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        tc::mma_bf16(tbase + (uint32_t)(128 + b * 64),
+                                                     tc::sdesc_add(dxa, (uint32_t)b * 128 * 128 + kk * 32),
+                                                     tc::sdesc_add(dbb, (uint32_t)p * 8192 + kk * 2048), idy,
+                                                     (k > 0 || p > 0 || kk > 0) ? 1u : 0u);
                         }
+                        tc::mma_commit(&mbar[3 + (pi & 1)]);
+                        if (k == c) tc::mma_commit(&mbar[5]);
                     }
-                }
-            }
-            if (!ok) break;
-            // G' complete; the last two stage commits are consumed so every commit has its wait
-            if (tid == 0) tc::mma_commit(&mbar[5]);
-            ok &= tc::mbar_wait(&mbar[5], phy, st);
-            phy ^= 1;
-            for (int q = 0; q < 2; ++q) {
-                ok &= tc::mbar_wait(&mbar[3 + q], phs[q], st);
-                phs[q] ^= 1;
-            }
-        }
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-
-        // ---------------- 16-column panels with a one-panel look-ahead
-        // Panel j: its 16 TMEM columns -> registers; the 16 x 16 diagonal block is factored by its
-        // half-warp with shuffles; every other live row solves its 16 values against it; the values
-        // are staged as three bf16 pieces (two staging buffers, alternating) and one thread issues
-        // the negated K = 16 tcgen05 MMAs of the trailing update in two groups: the next panel's 16
-        // columns (committed to mbar[0]) and then every later column (committed to mbar[1]).  Panel
-        // j+1 waits for mbar[0] only, so the bulk of the update runs under its factorization.  In
-        // the factor mode the rows of the diagonal block must start their B entries right of the
-        // panel from zero: the other warp of their TMEM lane group resets those entries once the
-        // previous panel's bulk update has landed, while the diagonal block is being factored.
-        __nv_bfloat16 *Bs = FACTOR ? Bscr + (size_t)s * 3 * D * D : nullptr;
-        const int npan = (n + 15) / 16;
-        // phase bookkeeping: panel j < npan - 1 commits once to each barrier; completion k of a
-        // barrier is awaited with parity (base + k) & 1
-        const uint32_t base0 = ph0, base1 = ph1;
-        for (int j = 0; j < npan; ++j) {
-            const int j0 = 16 * j;
-            const int nb = min(16, n - j0);
-            const int j1 = j0 + nb;
-            const int ii = row - j0;
-            const bool diag = ii >= 0 && ii < 16;
-            const uint32_t R = region + (uint32_t)(j & 1) * TmemChol::PANEL;
-            if (j > 0) {
-                // the previous panel's update of these 16 columns (and every earlier MMA) has landed;
-                // a timeout is acted on at the next block-wide vote
-                ok &= tc::mbar_wait(&mbar[0], (base0 + (uint32_t)(j - 1)) & 1u, st);
-                tc::fence_after_sync();
-            }
-            float v[16];
-            __syncwarp();
-            tc::tmem_ld16(trow + (uint32_t)j0, v);
-            const int gd = (j0 & 127) >> 5, bd = j0 >> 7;     // lane group, row block of the block rows
-            if (FACTOR && j1 < n && warp == (1 - bd) * 4 + gd) {   // warp-uniform: the reset helper
-                bool okh = true;
-                if (j > 0) {
-                    okh = tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(j - 1)) & 1u, st);   // previous bulk update
-                    tc::fence_after_sync();
-                }
-                okh = __all_sync(0xffffffffu, okh);
-                if (okh) {
-                    const int lrow = bd * 128 + gd * 32 + lane;   // row of this lane in those columns
-                    const bool zero = lrow >= j0 && lrow < j0 + 16;
-                    const uint32_t tb = tbase + ((uint32_t)(gd * 32) << 16) + (uint32_t)(bd * 256);
-#pragma unroll 1
-                    for (int c0 = j1; c0 < D; c0 += 64) {
-                        const int cnt = min(4, (D - c0) >> 4);      // warp-uniform
-                        uint32_t r4[4][16];
+                    if (k == c) {
+                        // Y_c complete (and with it every earlier MMA, so the pieces buffer is free)
+                        if (ok) ok = tc::mbar_wait(&mbar[5], phy, st);
+                        phy ^= 1;
+                        tc::fence_after_sync();
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (ok) {
+                            float a64[64];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (q < cnt) tc::tmem_ld16_nw(tb + (uint32_t)(c0 + 16 * q), r4[q]);
-                        tc::tmem_wait_ld();
+                            for (int q = 0; q < 4; ++q) {
+                                float v16[16];
+                                tc::tmem_ld16(tbase + ((uint32_t)lb << 16) + (uint32_t)(128 + blk * 64 + q * 16), v16);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            if (q < cnt) {
-                                float t16[16];
+                                for (int i = 0; i < 16; ++i) a64[q * 16 + i] = sc * v16[i];
+                            }
+                            stage_row(region, row, a64, nullptr, 0);
+                        }
+                        tc::fence_async_smem();
+                        tc::fence_before_sync();
+                        ok = cbar_and(ok);
+                        if (issuer && ok) {
+                            tc::fence_after_sync();
+                            const uint64_t dyp = tc::sdesc(region, 16, 1024);
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) t16[i] = zero ? 0.f : __uint_as_float(r4[q][i]);
-                                tc::tmem_st16(tb + (uint32_t)(c0 + 16 * q), t16);
+                            for (int pr = 0; pr < 6; ++pr) {
+                                const uint32_t pa = (uint32_t)pair_a(pr) * TmemChol::PIECE;
+                                const uint32_t pb = (uint32_t)pair_b(pr) * TmemChol::PIECE;
+#pragma unroll
+                                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        tc::mma_bf16(tbase + (uint32_t)(b * 256),
+                                                     tc::sdesc_add(dyp, pa + (uint32_t)b * 128 * 128 + kk * 32),
+                                                     tc::sdesc_add(dyp, pb + kk * 32), b == 0 ? idg0 : idg1,
+                                                     (c > 0 || pr > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
                     }
+                }
+                // G' complete; the last two stage commits are consumed so every commit has its wait
+                if (issuer) tc::mma_commit(&mbar[5]);
+                if (ok) ok = tc::mbar_wait(&mbar[5], phy, st);
+                phy ^= 1;
+                for (int q = 0; q < 2; ++q) {
+                    if (ok) ok = tc::mbar_wait(&mbar[3 + q], phs[q], st);
+                    phs[q] ^= 1;
+                }
+            }
+            tc::fence_before_sync();
+            ok = cbar_and(ok);
+            tc::fence_after_sync();
+
+            // ---------------- 16-column panels with a one-panel look-ahead
+            // Panel j: its 16 TMEM columns -> registers; the 16 x 16 diagonal block is factored by its
+            // half-warp with shuffles; every other live row solves its 16 values against it; the
+            // values are staged as three bf16 pieces (two staging buffers, alternating) and the issuing
+            // thread issues the negated K = 16 tcgen05 MMAs of the trailing update in two groups: the next panel's 16 columns (committed to mbar[0]) and then every later column
+            // (committed to mbar[1]).  Panel j+1 waits for mbar[0] only, so the bulk of the update
+            // runs under its factorization.  In the factor mode the rows of the diagonal block must
+            // start their B entries right of the panel from zero: the other warp of their TMEM lane
+            // group resets those entries once the previous panel's bulk update has landed, while the
+            // diagonal block is being factored.
+            const int npan = (n + 15) / 16;
+            // phase bookkeeping: panel j < npan - 1 commits once to each barrier; completion k of a
+            // barrier is awaited with parity (base + k) & 1
+            const uint32_t base0 = ph0, base1 = ph1;
+            for (int j = 0; j < npan; ++j) {
+                const int j0 = 16 * j;
+                const int nb = min(16, n - j0);
+                const int j1 = j0 + nb;
+                const int ii = row - j0;
+                const bool diag = ii >= 0 && ii < 16;
+                const uint32_t R = region + (uint32_t)(j & 1) * TmemChol::PANEL;
+                if (j > 0) {
+                    // the previous panel's update of these 16 columns (and every earlier MMA) has
+                    // landed; a timeout is acted on at the next vote
+                    if (ok) ok = tc::mbar_wait(&mbar[0], (base0 + (uint32_t)(j - 1)) & 1u, st);
+                    tc::fence_after_sync();
+                }
+                float v[16];
+                __syncwarp();
+                tc::tmem_ld16(trow + (uint32_t)j0, v);
+                const int gd = (j0 & 127) >> 5, bd = j0 >> 7;     // lane group, row block of the block rows
+                if (FACTOR && j1 < n && warp == (1 - bd) * 4 + gd) {   // warp-uniform: the reset helper
+                    bool okh = ok;
+                    if (j > 0 && okh) {
+                        okh = tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(j - 1)) & 1u, st);   // previous bulk update
+                        tc::fence_after_sync();
+                    }
+                    okh = __all_sync(0xffffffffu, okh);
+                    if (okh) {
+                        const int lrow = bd * 128 + gd * 32 + lane;   // row of this lane in those columns
+                        const bool zero = lrow >= j0 && lrow < j0 + 16;
+                        const uint32_t tb = tbase + ((uint32_t)(gd * 32) << 16) + (uint32_t)(bd * 256);
+#pragma unroll 1
+                        for (int c0 = j1; c0 < D; c0 += 32) {
+                            const int cnt = min(2, (D - c0) >> 4);      // warp-uniform
+                            uint32_t r4[2][16];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q)
+                                if (q < cnt) tc::tmem_ld16_nw(tb + (uint32_t)(c0 + 16 * q), r4[q]);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                if (q < cnt) {
+                                    float t16[16];
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i) t16[i] = zero ? 0.f : __uint_as_float(r4[q][i]);
+                                    tc::tmem_st16(tb + (uint32_t)(c0 + 16 * q), t16);
+                                }
+                            }
+                        }
+                        tc::tmem_wait_st();
+                    }
+                    ok &= okh;
+                }
+                if (FACTOR && diag) {
+                    // right of its diagonal a row carries B, which only receives contributions from
+                    // columns at or after its own: what earlier updates left there is dropped
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (c > ii) v[c] = 0.f;
+                }
+                float a[16];
+                if (diag) {
+                    // branch-free (selects only): the half-warp stays converged for its shuffles, and
+                    // the per-pivot work on the serial path is one broadcast, one rsqrt and one fma;
+                    // each lane keeps its own pivot's values and writes them afterwards
+                    const int lb0 = lane & 16;
+                    const unsigned mask = 0xFFFFu << lb0;
+                    float rl_mine = 1.f, e_mine = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const float e = __shfl_sync(mask, v[c], lb0 + c);   // excess of column c
+                        const float rlc = rsqrtf(1.f + e);
+                        const float li = v[c] * rlc;                        // L_ii,c for ii > c
+#pragma unroll
+                        for (int c2 = 0; c2 < 16; ++c2) {
+                            if (c2 > c) {
+                                const float w = __shfl_sync(mask, v[c], lb0 + c2);
+                                const float u = fmaf(-li, w * rlc, v[c2]);
+                                v[c2] = ii >= c2 ? u : v[c2];
+                            }
+                        }
+                        const bool piv = ii == c;
+                        v[c] = piv ? (1.f + e) * rlc : (ii > c ? li : v[c]);  // L_cc on the pivot row
+                        rl_mine = piv ? rlc : rl_mine;
+                        e_mine = piv ? e : e_mine;
+                    }
+                    s_rl[ii] = rl_mine;
+                    if (!FACTOR && ii < nb && ok && dcheck(start + j0 + ii < N, st))
+                        dR[start + j0 + ii] = 0.5f * log1pf(e_mine);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) s_LdT[c][ii] = c <= ii ? v[c] : 0.f;
+                }
+                ok = cbar_and(ok);
+                // rows at or above the block are finished in the in-segment mode
+                const bool live = FACTOR || ii >= 16;
+                if (live) {
+                    // right-looking solve against the diagonal block: a[m] is final once the columns
+                    // before m are applied; a diagonal-block row takes the B role (B_im = 0 for m < ii,
+                    // B_ii = 1/L_ii); rows above the block carry B, rows below L
+                    float rl[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 r4 = reinterpret_cast<const float4 *>(s_rl)[q];
+                        rl[4 * q] = r4.x; rl[4 * q + 1] = r4.y; rl[4 * q + 2] = r4.z; rl[4 * q + 3] = r4.w;
+                    }
+                    const float binv = diag ? 1.f / s_LdT[ii][ii] : 0.f;      // B_ii = 1 / L_ii (IEEE)
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        float am = v[m] * rl[m];
+                        if (diag && m <= ii) am = m == ii ? binv : 0.f;
+                        a[m] = am;
+                        const float4 *lr = reinterpret_cast<const float4 *>(&s_LdT[m][0]);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (4 * q + 3 > m) {
+                                const float4 l = lr[q];
+                                if (4 * q + 0 > m) v[4 * q + 0] = fmaf(-am, l.x, v[4 * q + 0]);
+                                if (4 * q + 1 > m) v[4 * q + 1] = fmaf(-am, l.y, v[4 * q + 1]);
+                                if (4 * q + 2 > m) v[4 * q + 2] = fmaf(-am, l.z, v[4 * q + 2]);
+                                v[4 * q + 3] = fmaf(-am, l.w, v[4 * q + 3]);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) a[m] = 0.f;
+                }
+                if (FACTOR) {
+                    // the panel's final values stay in TMEM (B right of the diagonal, zero left of it
+                    // in the block rows, L below); B leaves for global memory once, after the panels
+                    tc::tmem_st16(trow + (uint32_t)j0, a);
                     tc::tmem_wait_st();
                 }
-                ok &= okh;
+                if (j1 < n) {
+                    // the row's 16 values as three bf16 pieces: operand rows of the trailing update (L
+                    // for rows >= j1, B in the factor mode for rows < j1, zero in the in-segment mode)
+                    uint32_t hh[8], mm[8], ll[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) split3x2(a[2 * q], a[2 * q + 1], hh[q], mm[q], ll[q]);
+#pragma unroll
+                    for (int k8 = 0; k8 < 2; ++k8) {
+                        const uint32_t off = tc::kmajor_off(row, k8 * 8);
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(R + off), "r"(hh[4 * k8]),
+                                     "r"(hh[4 * k8 + 1]), "r"(hh[4 * k8 + 2]), "r"(hh[4 * k8 + 3])
+                                     : "memory");
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(R + TmemChol::PIECE + off),
+                                     "r"(mm[4 * k8]), "r"(mm[4 * k8 + 1]), "r"(mm[4 * k8 + 2]), "r"(mm[4 * k8 + 3])
+                                     : "memory");
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(R + 2 * TmemChol::PIECE + off),
+                                     "r"(ll[4 * k8]), "r"(ll[4 * k8 + 1]), "r"(ll[4 * k8 + 2]), "r"(ll[4 * k8 + 3])
+                                     : "memory");
+                    }
+                }
+                if (j1 < n) {
+                    tc::fence_async_smem();
+                    tc::fence_before_sync();
+                    ok = cbar_and(ok);                  // the whole panel is staged
+                    if (issuer) {
+                        const uint64_t dR_reg = tc::sdesc_add(dregion, (uint32_t)(j & 1) * TmemChol::PANEL);
+                        if (ok) {
+                            tc::fence_after_sync();
+                            // the next panel's 16 columns first, then everything right of them
+#pragma unroll
+                            for (int b = 0; b < 2; ++b) {
+                                if (!FACTOR && (b + 1) * 128 <= j1) continue;
+                                issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1), dR_reg, b * 128, j1,
+                                                    idesc_neg(16));
+                            }
+                        }
+                        tc::mma_commit(&mbar[0]);
+                        if (ok) {
+#pragma unroll
+                            for (int b = 0; b < 2; ++b) {
+                                if (!FACTOR && (b + 1) * 128 <= j1) continue;
+                                // in-segment mode: the first row block only needs its lower triangle
+                                const int nc = ((!FACTOR && b == 0) ? 128 : 256) - j1 - 16;
+                                if (nc > 0)
+                                    issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1 + 16), dR_reg, b * 128,
+                                                        j1 + 16, idesc_neg(nc));
+                            }
+                        }
+                        tc::mma_commit(&mbar[1]);
+                    }
+                }
             }
-            if (FACTOR && diag) {
-                // right of its diagonal a row carries B, which only receives contributions from
-                // columns at or after its own: what earlier updates left there is dropped
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    if (c > ii) v[c] = 0.f;
+            // every MMA of this segment has landed before the next segment (or the exit) reuses TMEM
+            if (npan > 1) {
+                if (ok) ok = tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(npan - 2)) & 1u, st);
+                tc::fence_after_sync();
             }
-            float a[16];
-            if (diag) {
-                // branch-free (selects only): the half-warp stays converged for its shuffles, and
-                // the per-pivot work on the serial path is one broadcast, one rsqrt and one fma;
-                // each lane keeps its own pivot's values and writes them afterwards
-                const int lb0 = lane & 16;
-                const unsigned mask = 0xFFFFu << lb0;
-                float rl_mine = 1.f, e_mine = 0.f;
+            ph0 = (base0 + (uint32_t)(npan - 1)) & 1u;
+            ph1 = (base1 + (uint32_t)(npan - 1)) & 1u;
+            ok = cbar_and(ok);
+            if (FACTOR && ok) {
+                // B = L^{-T} (TMEM upper triangle with the diagonal) -> three bf16 pieces in global
+                // memory, 64 columns at a time: each thread splits its row (zero left of the diagonal)
+                // into shared memory (row-major, 16-byte chunks XOR-swizzled by row), then warps copy
+                // whole 128-byte row pieces out.  Rows below a chunk's last panel are never read by the
+                // whitening loads and are not stored.
+                __nv_bfloat16 *Bs = Bscr + (size_t)s * 3 * D * D;
+                uint8_t *stg = smraw + (region - tc::smem_u32(smraw));
+#pragma unroll 1
+                for (int q = 0; q < D / 64; ++q) {
+#pragma unroll 1
+                    for (int h = 0; h < 4; ++h) {
+                        float v16[16];
+                        tc::tmem_ld16(trow + (uint32_t)(q * 64 + h * 16), v16);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float e = __shfl_sync(mask, v[c], lb0 + c);   // excess of column c
-                    const float rlc = rsqrtf(1.f + e);
-                    const float li = v[c] * rlc;                        // L_ii,c for ii > c
+                        for (int i = 0; i < 16; ++i)
+                            if (q * 64 + h * 16 + i < row) v16[i] = 0.f;
+                        uint32_t hh[8], mm[8], ll[8];
 #pragma unroll
-                    for (int c2 = 0; c2 < 16; ++c2) {
-                        if (c2 > c) {
-                            const float w = __shfl_sync(mask, v[c], lb0 + c2);
-                            const float u = fmaf(-li, w * rlc, v[c2]);
-                            v[c2] = ii >= c2 ? u : v[c2];
+                        for (int k = 0; k < 8; ++k) split3x2(v16[2 * k], v16[2 * k + 1], hh[k], mm[k], ll[k]);
+#pragma unroll
+                        for (int c2 = 0; c2 < 2; ++c2) {
+                            const int ch = (h * 2 + c2) ^ (row & 7);
+                            const size_t o = (size_t)row * 128 + ch * 16;
+                            *reinterpret_cast<uint4 *>(stg + o) =
+                                make_uint4(hh[4 * c2], hh[4 * c2 + 1], hh[4 * c2 + 2], hh[4 * c2 + 3]);
+                            *reinterpret_cast<uint4 *>(stg + 256 * 128 + o) =
+                                make_uint4(mm[4 * c2], mm[4 * c2 + 1], mm[4 * c2 + 2], mm[4 * c2 + 3]);
+                            *reinterpret_cast<uint4 *>(stg + 2 * 256 * 128 + o) =
+                                make_uint4(ll[4 * c2], ll[4 * c2 + 1], ll[4 * c2 + 2], ll[4 * c2 + 3]);
                         }
                     }
-                    const bool piv = ii == c;
-                    v[c] = piv ? (1.f + e) * rlc : (ii > c ? li : v[c]);  // L_cc on the pivot row
-                    rl_mine = piv ? rlc : rl_mine;
-                    e_mine = piv ? e : e_mine;
-                }
-                s_rl[ii] = rl_mine;
-                if (!FACTOR && ii < nb && dcheck(start + j0 + ii < N, st)) dR[start + j0 + ii] = 0.5f * log1pf(e_mine);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) s_LdT[c][ii] = c <= ii ? v[c] : 0.f;
-            }
-            ok = __syncthreads_and(ok) != 0;
-            if (!ok) break;
-            // rows at or above the block are finished in the in-segment mode
-            const bool live = FACTOR || ii >= 16;
-            if (live) {
-                // right-looking solve against the diagonal block: a[m] is final once the columns
-                // before m are applied; a diagonal-block row takes the B role (B_im = 0 for m < ii,
-                // B_ii = 1/L_ii); rows above the block carry B, rows below L
-                float rl[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 r4 = reinterpret_cast<const float4 *>(s_rl)[q];
-                    rl[4 * q] = r4.x; rl[4 * q + 1] = r4.y; rl[4 * q + 2] = r4.z; rl[4 * q + 3] = r4.w;
-                }
-                const float binv = diag ? 1.f / s_LdT[ii][ii] : 0.f;      // B_ii = 1 / L_ii (IEEE)
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    float am = v[m] * rl[m];
-                    if (diag && m <= ii) am = m == ii ? binv : 0.f;
-                    a[m] = am;
-                    const float4 *lr = reinterpret_cast<const float4 *>(&s_LdT[m][0]);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (4 * q + 3 > m) {
-                            const float4 l = lr[q];
-                            if (4 * q + 0 > m) v[4 * q + 0] = fmaf(-am, l.x, v[4 * q + 0]);
-                            if (4 * q + 1 > m) v[4 * q + 1] = fmaf(-am, l.y, v[4 * q + 1]);
-                            if (4 * q + 2 > m) v[4 * q + 2] = fmaf(-am, l.z, v[4 * q + 2]);
-                            v[4 * q + 3] = fmaf(-am, l.w, v[4 * q + 3]);
-                        }
+                    cbar();
+                    const int nrows = min(D, q * 64 + 64);                 // rows that hold B in this chunk
+                    for (int e = tid; e < 3 * nrows * 8; e += 256) {
+                        const int p = e / (nrows * 8), rest = e - p * nrows * 8, r = rest >> 3, c = rest & 7;
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stg + (size_t)p * 256 * 128 + (size_t)r * 128 +
+                                                                           ((c ^ (r & 7)) * 16));
+                        *reinterpret_cast<uint4 *>(Bs + (size_t)p * D * D + (size_t)r * D + q * 64 + c * 8) = val;
                     }
-                }
-            } else {
-#pragma unroll
-                for (int m = 0; m < 16; ++m) a[m] = 0.f;
-            }
-            if (FACTOR && row < j1) {
-                // B panel -> global pieces (rows >= j1 are zero here and never stored: the loads
-                // of the whitening GEMM zero-fill them)
-                __nv_bfloat16 *g = Bs + (size_t)row * D + j0;
-#pragma unroll
-                for (int k8 = 0; k8 < 2; ++k8) {
-                    uint32_t hh[4], mm[4], ll[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint16_t h0, m0, l0, h1, m1, l1;
-                        split3v(a[k8 * 8 + 2 * q], h0, m0, l0);
-                        split3v(a[k8 * 8 + 2 * q + 1], h1, m1, l1);
-                        hh[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                        mm[q] = (uint32_t)m0 | ((uint32_t)m1 << 16);
-                        ll[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-                    }
-                    *reinterpret_cast<uint4 *>(g + k8 * 8) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
-                    *reinterpret_cast<uint4 *>(g + (size_t)D * D + k8 * 8) = make_uint4(mm[0], mm[1], mm[2], mm[3]);
-                    *reinterpret_cast<uint4 *>(g + (size_t)2 * D * D + k8 * 8) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
-                }
-            }
-            if (j1 < n) {
-                // operand rows of the trailing update: L (rows >= j1), B (factor mode, rows < j1),
-                // zero (in-segment mode, rows < j1)
-                stage_row16(R, row, a);
-            }
-            tc::fence_async_smem();
-            tc::fence_before_sync();
-            __syncthreads();
-            if (j1 < n) {
-                if (tid == 0) {
-                    tc::fence_after_sync();
-                    // the next panel's 16 columns first, then everything right of them
-#pragma unroll
-                    for (int b = 0; b < 2; ++b) {
-                        if (!FACTOR && (b + 1) * 128 <= j1) continue;
-                        issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1), R, b * 128, j1, idesc_neg(16));
-                    }
-                    tc::mma_commit(&mbar[0]);
-#pragma unroll
-                    for (int b = 0; b < 2; ++b) {
-                        if (!FACTOR && (b + 1) * 128 <= j1) continue;
-                        // in-segment mode: the first row block only needs its lower triangle (columns < 128)
-                        const int nc = ((!FACTOR && b == 0) ? 128 : 256) - j1 - 16;
-                        if (nc > 0)
-                            issue_split_mma_k16(tbase + (uint32_t)(b * 256 + j1 + 16), R, b * 128, j1 + 16,
-                                                idesc_neg(nc));
-                    }
-                    tc::mma_commit(&mbar[1]);
+                    cbar();
                 }
             }
         }
-        // every MMA of this segment has landed before the next segment (or the exit) reuses TMEM
-        if (ok && npan > 1) {
-            ok &= tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(npan - 2)) & 1u, st);
-            tc::fence_after_sync();
-        }
-        ph0 = (base0 + (uint32_t)(npan - 1)) & 1u;
-        ph1 = (base1 + (uint32_t)(npan - 1)) & 1u;
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-
     }
-    if (tid == 0) {
+    tc::fence_before_sync();
+    __syncthreads();
+    if (issuer) {
         // MMAs still in flight (only after a timeout) finish before the tensor memory is freed
+        // (a commit tracks the MMAs of the thread that issued them)
         tc::mma_commit(&mbar[2]);
         tc::mbar_wait(&mbar[2], 0, st);
     }

@@ -5,13 +5,23 @@
 // positions with the largest dR among t >= 1 join it, and the K boundaries are
 // listed in time order.  Ties are broken towards the earlier position.
 //
-// One CTA per row: the row's dR values become order-preserving 32-bit keys
+// Rows of up to kClusterKeys candidates (all the workloads' rows) are selected
+// by a cluster of kCluster CTAs per row, each holding a contiguous slice of the
+// row's keys in shared memory: every radix pass builds the slice histograms,
+// each CTA reads the others' histograms through distributed shared memory
+// (plain loads, no multicast) and takes the same decision, and the ordered
+// compaction offsets each slice by the counts of the slices before it.
+// Longer rows take one CTA per row: the row's dR values become order-preserving 32-bit keys
 // (in shared memory when they fit), a 4-pass 8-bit radix select finds the
 // (K-1)-th largest key v and how many keys equal to v are still needed (the
 // histogram increments are aggregated per warp: the keys of a row share their
 // leading bytes), and one ordered pass writes the selected positions, which are
 // then already in increasing order (no sort).
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace dbc {
 namespace tk {
@@ -265,6 +275,173 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float *__restric
     }
 }
 
+
+// ---------------------------------------------------------------- cluster per row
+constexpr int kCluster = 8;
+constexpr int kCThreads = 256;
+constexpr int kCWarps = kCThreads / 32;
+constexpr int kSliceKeys = 8192;                       // keys per CTA slice (32 KB)
+constexpr int kClusterKeys = kCluster * kSliceKeys;    // candidates per row on this path
+constexpr int kWarpKeys = kSliceKeys / kCWarps;       // keys of a slice per warp (1024)
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
+    select_cluster_kernel(const float *__restrict__ dR, const int64_t *offsets, int64_t rows, int64_t T,
+                          const int64_t *Kp, int64_t Ks, int64_t dense_K, int64_t *idx_offsets, int64_t *idx,
+                          int32_t *st) {
+    __shared__ uint32_t keys[kSliceKeys];
+    __shared__ uint32_t hist[2][256];                  // alternate passes: a pass never clears what is read
+    __shared__ uint32_t tot[256];
+    __shared__ uint32_t s_bin;
+    __shared__ int s_rem;
+    __shared__ int s_cnt[2];                           // this slice's equal-key and selected counts
+    __shared__ int s_weq[kCWarps], s_wsel[kCWarps];    // per-warp counts, then their exclusive prefix
+    cg::cluster_group cluster = cg::this_cluster();
+    const int q = (int)cluster.block_rank();
+    const int64_t r = blockIdx.x / kCluster;
+    const int tid = threadIdx.x;
+    // every decision below is uniform over the cluster (it depends on the row only)
+    int64_t a, n;
+    row_bounds(offsets, r, T, a, n);
+    const int64_t K = row_K(Kp, Ks, r, nullptr);
+    int64_t obase;
+    if (dense_K > 0) {
+        const int64_t per = T < dense_K ? T : dense_K;
+        obase = r * per;
+        if (q == 0 && tid == 0) {
+            idx_offsets[r] = obase;
+            if (r == rows - 1) idx_offsets[rows] = rows * per;
+        }
+    } else {
+        obase = idx_offsets[r];
+    }
+    int64_t *out = idx + obase;
+    if (n <= 0) return;
+    if (K >= n) {
+        for (int64_t t = (int64_t)q * kCThreads + tid; t < n; t += kCluster * kCThreads) out[t] = t;
+        return;
+    }
+    if (q == 0 && tid == 0) out[0] = 0;
+    const int need = (int)(K - 1);
+    if (need == 0) return;
+    const int m = (int)(n - 1);                        // candidates t = 1 .. n-1 (m <= kClusterKeys)
+    const int slice = (m + kCluster - 1) / kCluster;
+    const int k0 = q * slice, k1 = min(m, k0 + slice); // this CTA's candidates [k0, k1)
+    const int mine = max(0, k1 - k0);
+    const float *row = dR + a + 1;
+    bool bad = false;
+    for (int j = tid; j < mine; j += kCThreads) {
+        const float f = row[k0 + j];
+        bad |= !isfinite(f);
+        keys[j] = key_of(f);
+    }
+    if (bad) flag(st, DBC_ERR_NONFINITE);
+    uint32_t prefix = 0, mask = 0;
+    int rem = need;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        uint32_t *h = hist[pass & 1];
+        h[tid] = 0;                                    // kCThreads == 256 bins
+        __syncthreads();
+        for (int base = 0; base < mine; base += kCThreads) {     // uniform trip count: whole warps
+            const int j = base + tid;
+            const uint32_t k = j < mine ? keys[j] : 0u;
+            hist_add(h, j < mine && (k & mask) == prefix, (k >> shift) & 255u);
+        }
+        cluster.sync();                                // every slice's histogram is complete
+        uint32_t total = 0;
+#pragma unroll
+        for (int c = 0; c < kCluster; ++c) total += cluster.map_shared_rank(h, c)[tid];
+        tot[tid] = total;
+        __syncthreads();
+        if (tid < 32) {
+            // warp 0: suffix sums over 8 bins per lane (from the top bin down), then pick the bin
+            uint32_t c8[8];
+            uint32_t loc = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) { c8[b] = tot[255 - (tid * 8 + b)]; loc += c8[b]; }
+            uint32_t inc = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (tid >= o) inc += y;
+            }
+            const uint32_t before = inc - loc;
+            if ((int)before < rem && (int)inc >= rem) {
+                uint32_t cum = before;
+#pragma unroll
+                for (int b = 0; b < 8; ++b) {
+                    if ((int)(cum + c8[b]) >= rem) {
+                        s_bin = 255u - (uint32_t)(tid * 8 + b);
+                        s_rem = rem - (int)cum;
+                        break;
+                    }
+                    cum += c8[b];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= s_bin << shift;
+        mask |= 255u << shift;
+        rem = s_rem;
+    }
+    // ordered compaction: key > v, or key == v among the first `rem` equal keys of the row.  Warp w
+    // owns keys [w * kWarpKeys, (w + 1) * kWarpKeys) of the slice and walks them 32 at a time (lane l
+    // takes key step * 32 + l: conflict-free shared loads), ranking with ballots; warps are offset by
+    // the warps before them, slices by the slices before them.
+    const uint32_t v = prefix;
+    const int lane = tid & 31, wid = tid >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    const int wk0 = wid * kWarpKeys;
+    int n_eq = 0, n_gt = 0;                            // warp totals (every lane holds them)
+    for (int step = 0; step < kWarpKeys / 32; ++step) {
+        const int j = wk0 + step * 32 + lane;
+        const uint32_t k = j < mine ? keys[j] : 0u;
+        n_eq += __popc(__ballot_sync(0xffffffffu, j < mine && k == v));
+        n_gt += __popc(__ballot_sync(0xffffffffu, j < mine && k > v));
+    }
+    if (lane == 0) {
+        s_weq[wid] = n_eq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int c = 0;
+        for (int w = 0; w < kCWarps; ++w) { const int x = s_weq[w]; s_weq[w] = c; c += x; }
+        s_cnt[0] = c;                                  // equal keys of the slice
+    }
+    cluster.sync();
+    int eq_before = s_weq[wid];
+    for (int c = 0; c < q; ++c) eq_before += cluster.map_shared_rank(s_cnt, c)[0];
+    const int left = rem - eq_before;
+    const int take_eq = left <= 0 ? 0 : (left >= n_eq ? n_eq : left);
+    if (lane == 0) s_wsel[wid] = n_gt + take_eq;
+    __syncthreads();
+    if (tid == 0) {
+        int c = 0;
+        for (int w = 0; w < kCWarps; ++w) { const int x = s_wsel[w]; s_wsel[w] = c; c += x; }
+        s_cnt[1] = c;                                  // selected keys of the slice
+    }
+    cluster.sync();
+    int sel_before = s_wsel[wid];
+    for (int c = 0; c < q; ++c) sel_before += cluster.map_shared_rank(s_cnt, c)[1];
+    int64_t o = 1 + (int64_t)sel_before;
+    int eq_run = 0;
+    for (int step = 0; step < kWarpKeys / 32; ++step) {
+        const int j = wk0 + step * 32 + lane;
+        const uint32_t k = j < mine ? keys[j] : 0u;
+        const bool eq = j < mine && k == v;
+        const unsigned em = __ballot_sync(0xffffffffu, eq);
+        const bool sel = (j < mine && k > v) || (eq && eq_run + __popc(em & lt) < take_eq);
+        const unsigned sm = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+            const int64_t at = o + __popc(sm & lt);
+            if (dcheck(at <= need, st)) out[at] = k0 + j + 1;
+        }
+        o += __popc(sm);
+        eq_run += __popc(em);
+    }
+    cluster.sync();                                    // no CTA leaves while its counts may still be read
+}
+
 }  // namespace tk
 }  // namespace dbc
 
@@ -296,6 +473,13 @@ extern "C" dbc_status chunk_topk_select(const float *dR, const int64_t *offsets,
     }
     if (rows == 0 || N == 0) return launch_status();
     const int64_t m = T > 1 ? T - 1 : 1;
+    if (m <= tk::kClusterKeys && rows <= INT32_MAX / tk::kCluster) {
+        // every row fits the cluster path (T is the longest row)
+        tk::select_cluster_kernel<<<(unsigned)(rows * tk::kCluster), tk::kCThreads, 0, s>>>(
+            dR, offsets, rows, T, K_per_row, K_scalar, dense_K, idx_offsets, idx, dev_status);
+        count_launches(1);
+        return launch_status();
+    }
     const int keys = (int)std::min<int64_t>(m, tk::kSmemKeys);
     const size_t smem = (size_t)keys * sizeof(uint32_t);
     cudaFuncSetAttribute(tk::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

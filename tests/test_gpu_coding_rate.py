@@ -181,12 +181,13 @@ def test_topk_bit_exact_on_gpu_dR():
         assert np.array_equal(idx[io[r]:io[r + 1]], want), r
 
 
-def test_topk_large_rows_from_global_memory():
-    """Rows longer than the shared-memory key buffer take the global-memory path."""
+@pytest.mark.parametrize("T,K", [(70000, 9000), (65537, 20000), (60000, 7), (49153, 30000)])
+def test_topk_large_rows_from_global_memory(T, K):
+    """Long rows: up to 65536 candidates the per-row CTA cluster (slices of up to 8192 keys in each
+    CTA's shared memory), beyond that one CTA per row reading the keys from global memory."""
     import torch
     import dynamic_byte_chunking_b200 as dbc
     rng = np.random.default_rng(4)
-    T, K = 70000, 9000
     vals = rng.random(2 * T).astype(np.float32)
     vals[::7] = 0.5
     d = torch.from_numpy(vals).cuda()
