@@ -51,6 +51,10 @@ def parse():
     ap.add_argument("--reps", type=int, default=10)
     ap.add_argument("--families", default="tiny,byteflow,bytegen,wide,ragged",
                     help="workload families measured by --rows (comma-separated)")
+    ap.add_argument("--probe", default=None, metavar="FAMILY",
+                    help="run the path twice on one workload family (coding rate, Top-K, gather, upsample, and the "
+                         "router with EMA where the family has router weights), check the device status and exit: "
+                         "a short, fixed launch sequence for profilers")
     ap.add_argument("--traffic-from", default=None, metavar="CSV",
                     help="convert an ncu --csv launch list with dram__bytes_read.sum and dram__bytes_write.sum "
                          "(taken on this workload) into profiles/dram_traffic_byteflow.json, then exit")
@@ -463,11 +467,49 @@ def run_rows(args):
         torch.cuda.empty_cache()
 
 
+def run_probe(family, reps=2):
+    """The path `reps` times on one family, in a fixed launch order (for ncu -k / -s / -c)."""
+    import torch
+    import workloads
+    import dynamic_byte_chunking_b200 as dbc
+    dev = torch.device("cuda", 0)
+    w = workloads.make(family)
+    H = torch.from_numpy(w.H_bits.view(np.int16)).view(torch.bfloat16).to(dev) if w.dtype == "bf16" else \
+        torch.from_numpy(w.H_bits).to(dev)
+    rows, T, d, N = w.rows, w.T, w.d, w.N
+    o = None if w.dense else torch.from_numpy(w.offsets).to(dev)
+    Hx = H.view(rows, T, d) if w.dense else H
+    Kt = torch.from_numpy(w.K).to(dev)
+    total = int(np.minimum(w.K, w.lengths).sum())
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(dbc.chunk_coding_rate_workspace(rows, T, N, d), dtype=torch.uint8, device=dev)
+    dR = torch.empty(N, dtype=torch.float32, device=dev)
+    Wb = (torch.from_numpy(w.W_bin.view(np.int16)).view(torch.bfloat16).to(dev)
+          if w.W_bin is not None and w.W_proj is None else None)
+    Wq = torch.from_numpy(w.Wq.view(np.int16)).view(torch.bfloat16).to(dev) if w.Wq is not None else None
+    Wk = torch.from_numpy(w.Wk.view(np.int16)).view(torch.bfloat16).to(dev) if w.Wk is not None else None
+    for _ in range(reps):
+        dbc.chunk_coding_rate(Hx, w.eps2, offsets=o, T=T, dR=dR, workspace=ws, dev_status=st)
+        idx, io = dbc.chunk_topk_select(dR, Kt, rows=rows, T=T, offsets=o, total=total, dev_status=st)
+        Z = dbc.chunk_gather(H, idx, io, rows=rows, T=T, offsets=o, total=total, dev_status=st)
+        if Wb is not None:
+            dbc.chunk_upsample(Z, H, idx, io, Wb, rows=rows, T=T, offsets=o, dev_status=st)
+        if Wq is not None:
+            dbc.hnet_route(Hx, Wq, Wk, offsets=o, T=T, do_ema=True, dev_status=st)
+    torch.cuda.synchronize()
+    if st.item() != 0:
+        raise RuntimeError(f"device status flags {st.item():#x}")
+    print(json.dumps({"probe": family, "reps": reps, "launches": dbc.launch_count()}))
+
+
 # ---------------------------------------------------------------- device arm
 def main():
     args = parse()
     if args.traffic_from:
         write_traffic(args.traffic_from)
+        return
+    if args.probe:
+        run_probe(args.probe)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -17,7 +17,9 @@
 //     segment's MMAs overlap this segment's epilogue;
 //   * eight epilogue warps read the tile from TMEM, store c * (running sum)
 //     as P_s (fp32, the exclusive prefix) and add G_s to the running sum,
-//     which each thread keeps in float64 registers for its row and columns.
+//     which each thread keeps for its row and columns as a compensated fp32
+//     pair (hi + lo, about 48 significant bits: every addition's exact error
+//     is carried in lo), as accurate here as float64 and far cheaper.
 // The running sum may start from a carried float64 state (streams) and is
 // then written back (the whole symmetric matrix: off-diagonal tiles also
 // write their transpose).  Every mbarrier wait is bounded; a role that gives up
@@ -185,14 +187,21 @@ __global__ void __launch_bounds__(GramPrefixCfg<TN>::NT, 1) gram_prefix_kernel(
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue: running float64 sums of this thread's row and columns
+        // ---------------- epilogue: running sums of this thread's row and columns, each kept as an
+        // unevaluated fp32 pair hi + lo (compensated summation, ~48 significant bits: the exact
+        // error of every fp32 addition is carried in lo), much cheaper than float64 arithmetic
         const int lg = warp & 3, half = (warp - 2) >> 2;
         const int f1 = b * 128 + lg * 32 + lane;
         const int f2 = n * TN + half * C::CPT;
-        double acc[C::CPT];
+        float hi[C::CPT], lo[C::CPT];
         double *srow = state ? state + ((size_t)r * D + f1) * D + f2 : nullptr;
 #pragma unroll
-        for (int i = 0; i < C::CPT; ++i) acc[i] = srow ? srow[i] : 0.0;
+        for (int i = 0; i < C::CPT; ++i) {
+            const double s0v = srow ? srow[i] : 0.0;
+            hi[i] = (float)s0v;
+            lo[i] = (float)(s0v - (double)hi[i]);
+        }
+        const float cf = (float)c;
         bool ok = true, bad = false;
         int seg_i = 0;
         for (int s = s0; s < s1; ++s, ++seg_i) {
@@ -208,15 +217,23 @@ __global__ void __launch_bounds__(GramPrefixCfg<TN>::NT, 1) gram_prefix_kernel(
                                  u);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[q * 4 + i] = make_float4((float)(c * acc[q * 16 + 4 * i]), (float)(c * acc[q * 16 + 4 * i + 1]),
-                                                 (float)(c * acc[q * 16 + 4 * i + 2]),
-                                                 (float)(c * acc[q * 16 + 4 * i + 3]));
+                for (int i4 = 0; i4 < 4; ++i4) {
+                    float pv[4];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float v = __uint_as_float(u[i]);
-                    bad |= !isfinite(v);
-                    acc[q * 16 + i] += (double)v;
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = q * 16 + i4 * 4 + e;
+                        pv[e] = __fadd_rn(__fmul_rn(cf, hi[i]), __fmul_rn(cf, lo[i]));
+                        const float v = __uint_as_float(u[i4 * 4 + e]);
+                        bad |= !isfinite(v);
+                        // two-sum: hi + v = sum + err exactly
+                        const float h = hi[i];
+                        const float sum = __fadd_rn(h, v);
+                        const float bv = __fsub_rn(sum, h);
+                        const float err = __fadd_rn(__fsub_rn(h, __fsub_rn(sum, bv)), __fsub_rn(v, bv));
+                        hi[i] = sum;
+                        lo[i] = __fadd_rn(lo[i], err);
+                    }
+                    dst[q * 4 + i4] = make_float4(pv[0], pv[1], pv[2], pv[3]);
                 }
             }
             tc::fence_before_sync();
@@ -226,12 +243,12 @@ __global__ void __launch_bounds__(GramPrefixCfg<TN>::NT, 1) gram_prefix_kernel(
         if (bad) flag(st, DBC_ERR_NONFINITE);
         if (srow && ok) {
 #pragma unroll
-            for (int i = 0; i < C::CPT; ++i) srow[i] = acc[i];
+            for (int i = 0; i < C::CPT; ++i) srow[i] = (double)hi[i] + (double)lo[i];
             if (!diag) {
                 // the carried state is the whole symmetric matrix: mirror the off-diagonal block
                 double *scol = state + (size_t)r * D * D + f1;
-#pragma unroll 1
-                for (int i = 0; i < C::CPT; ++i) scol[(size_t)(f2 + i) * D] = acc[i];
+#pragma unroll
+                for (int i = 0; i < C::CPT; ++i) scol[(size_t)(f2 + i) * D] = (double)hi[i] + (double)lo[i];
             }
         }
     }

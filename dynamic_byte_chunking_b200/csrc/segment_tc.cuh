@@ -474,27 +474,23 @@ namespace dbc {
 namespace cr {
 
 // P_s = c (state + the row's earlier segment Grams) for every segment, through the fused TMA-fed
-// Gram + float64 prefix kernel (one CTA per row and 128 x TN tile).  Returns false (nothing
+// Gram + prefix kernel (one CTA per row and 128 x 64 tile).  Returns false (nothing
 // launched) when the row count and lengths favour the segment-parallel Gram and prefix kernels,
 // or when no tensor map can be encoded.
 inline bool launch_gram_prefix(const __nv_bfloat16 *H, int64_t N, int64_t rows, int64_t ns, const Segs &segs,
                                float *P, double *state, double c, int32_t *st, cudaStream_t stream) {
     const int sms = num_sms();
-    // few long rows leave most SMs idle in a per-row walk
-    if (rows * 6 < sms && ns > rows * 128) return false;
+    // Each CTA walks its row's segments one after another (about 3 us a segment), so with fewer
+    // CTAs than half the SMs the segment-parallel Gram kernel and the prefix kernel finish first
+    // (8 rows of 8192 positions: 61 us against 100 us; 64 rows of 4096: 252 us against 158 us).
+    if (rows * GramPrefixCfg<64>::TILES * 2 < sms && ns > rows * 2) return false;
     if (rows * 6 > INT32_MAX / 2) return false;
     CUtensorMap tm;
     if (!tma::encode_bf16_rows(&tm, H, (uint64_t)N, 256, 64)) return false;
-    if (rows * 6 <= 2 * (int64_t)sms) {
-        using C = GramPrefixCfg<64>;
-        cudaFuncSetAttribute(gram_prefix_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-        gram_prefix_kernel<64><<<(unsigned)(rows * C::TILES), C::NT, C::SMEM, stream>>>(tm, segs, rows, P, state, c, st);
-    } else {
-        using C = GramPrefixCfg<128>;
-        cudaFuncSetAttribute(gram_prefix_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-        gram_prefix_kernel<128><<<(unsigned)(rows * C::TILES), C::NT, C::SMEM, stream>>>(tm, segs, rows, P, state, c,
-                                                                                        st);
-    }
+    // 128 x 64 tiles: 32 running sums per epilogue thread (wider tiles would spill registers)
+    using C = GramPrefixCfg<64>;
+    cudaFuncSetAttribute(gram_prefix_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    gram_prefix_kernel<64><<<(unsigned)(rows * C::TILES), C::NT, C::SMEM, stream>>>(tm, segs, rows, P, state, c, st);
     return true;
 }
 
