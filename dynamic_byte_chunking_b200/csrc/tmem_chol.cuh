@@ -33,6 +33,14 @@
 namespace dbc {
 namespace cr {
 
+// 1 / sqrt(x) from the hardware approximation with subnormals flushed: the pivots are 1 + e with
+// e >= 0 in exact arithmetic, so the argument is never subnormal and the flush costs nothing.
+__device__ __forceinline__ float rsqrt_ftz(float x) {
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 struct TmemChol {
     static constexpr int NT = 256;
     static constexpr uint32_t PIECE = 256 * 128;          // 256-row x 64-K bf16 tile
@@ -135,8 +143,9 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     int64_t N, float c_rate, float *dR, int32_t *st) {
     constexpr int D = 256;
     extern __shared__ uint8_t smraw[];
-    // [0], [1] panel MMA groups; [2] the final drain; [3], [4] Y operand stages consumed; [5] Y chunk done
-    __shared__ uint64_t mbar[6];
+    // [0], [1] panel MMA groups; [2] the final drain; [3], [4] Y operand stages consumed; [5] Y chunk done;
+    // [6], [7] Y operand stages loaded (one arrival from each of the 224 loading threads)
+    __shared__ uint64_t mbar[8];
     __shared__ uint32_t tmem_base;
     __shared__ __align__(16) float s_LdT[16][16];   // factored 16 x 16 diagonal block, column-major
     __shared__ __align__(16) float s_rl[16];        // 1 / L_kk of the diagonal block
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) tc::mbar_init(&mbar[i], 1);
+        for (int i = 6; i < 8; ++i) tc::mbar_init(&mbar[i], 7 * 32);
         tc::fence_mbar_init();
     }
     tc::fence_before_sync();
@@ -168,7 +178,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
         // ================= thread (warp w, lane l) owns row (w/4)*128 + (w%4)*32 + l
         const uint32_t trow = tbase + ((uint32_t)lb << 16) + (uint32_t)(blk * 256);
         uint32_t ph0 = 0, ph1 = 0;      // mbarrier phases (uniform across the compute threads)
-        uint32_t phs[2] = {0, 0}, phy = 0;
+        uint32_t phs = 0, phy = 0, pf = 0;   // phs, pf: bit q = parity of the next wait on stage q
         bool ok = true;
         // A timeout makes `ok` false: every later wait and MMA is skipped (commits still arrive),
         // and the block-wide votes keep all threads on the same path to the end.
@@ -217,7 +227,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 auto load = [&](int pi, uint32_t sa) {
                     int c, k;
                     ypair(pi, c, k);
-                    for (int e = tid; e < 256 * 8; e += 256) {              // X: 256 positions x 64 K
+                    for (int e = tid; e < 256 * 8; e += 7 * 32) {           // X: 256 positions x 64 K
                         const int r = e >> 3, ch = e & 7;
                         const bool in = r < len;
                         const uint32_t xo =
@@ -225,7 +235,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                         tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + k * 64 + ch * 8, in ? 16u : 0u);
                     }
                     const uint32_t sb = sa + TmemChol::YX_BYTES;
-                    for (int e = tid; e < 3 * 64 * 8; e += 256) {           // B: 3 pieces x 64 K x 64 N
+                    for (int e = tid; e < 3 * 64 * 8; e += 7 * 32) {        // B: 3 pieces x 64 K x 64 N
                         const int p = e >> 9, kr = (e >> 3) & 63, n8 = e & 7;
                         const int krow = k * 64 + kr, col = c * 64 + n8 * 8;
                         const bool nz = krow < (col >> 4) * 16 + 16;         // stored rows of the columns' panel
@@ -234,7 +244,11 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     }
                 };
                 const float sc = sqrtf(c_rate);
-                load(0, region + TmemChol::YSTAGE0);
+                // warps 0..6 stream the operand stages and announce each on full[stage]; warp 7 only
+                // issues (its lane 0) and joins the Y_c read-outs, so a long MMA issue (G' takes a
+                // few thousand cycles) never holds up the next stage's loads
+                const bool loader = warp < 7;
+                if (loader) load(0, region + TmemChol::YSTAGE0);
                 tc::cp_async_commit();
                 for (int pi = 0; pi < NPAIR; ++pi) {
                     int c, k;
@@ -242,16 +256,20 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     if (pi + 1 < NPAIR) {
                         const int q = (pi + 1) & 1;
                         if (pi + 1 >= 2) {                                   // stage q was read by pair pi - 1
-                            if (ok) ok = tc::mbar_wait(&mbar[3 + q], phs[q], st);
-                            phs[q] ^= 1;
+                            if (loader && ok) ok = tc::mbar_wait(&mbar[3 + q], (phs >> q) & 1u, st);
+                            phs ^= 1u << q;
                         }
-                        load(pi + 1, region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE);
+                        if (loader) load(pi + 1, region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE);
                     }
                     tc::cp_async_commit();
-                    tc::cp_async_wait<1>();
-                    tc::fence_async_smem();
-                    ok = cbar_and(ok);                                       // stage pi complete everywhere
+                    if (loader) {
+                        tc::cp_async_wait<1>();
+                        tc::fence_async_smem();
+                        tc::mbar_arrive(&mbar[6 + (pi & 1)]);            // stage pi is in place
+                    }
                     if (issuer) {
+                        if (ok) ok = tc::mbar_wait(&mbar[6 + (pi & 1)], (pf >> (pi & 1)) & 1u, st);
+                        pf ^= 1u << (pi & 1);
                         if (ok) {
                             tc::fence_after_sync();
                             const uint32_t sa = region + TmemChol::YSTAGE0 + (uint32_t)(pi & 1) * TmemChol::YSTAGE;
@@ -315,8 +333,8 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 if (ok) ok = tc::mbar_wait(&mbar[5], phy, st);
                 phy ^= 1;
                 for (int q = 0; q < 2; ++q) {
-                    if (ok) ok = tc::mbar_wait(&mbar[3 + q], phs[q], st);
-                    phs[q] ^= 1;
+                    if (ok) ok = tc::mbar_wait(&mbar[3 + q], (phs >> q) & 1u, st);
+                    phs ^= 1u << q;
                 }
             }
             tc::fence_before_sync();
@@ -396,29 +414,48 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 }
                 float a[16];
                 if (diag) {
-                    // branch-free (selects only): the half-warp stays converged for its shuffles, and
-                    // the per-pivot work on the serial path is one broadcast, one rsqrt and one fma;
-                    // each lane keeps its own pivot's values and writes them afterwards
+                    // Two pivots per step (branch-free, selects only, so the half-warp stays converged
+                    // for its shuffles): the 2 x 2 diagonal block of columns (c, c+1) is factored
+                    // from three broadcasts taken at once, and both columns are applied to the rest
+                    // of the row together, so the serial path per pivot pair is one round of
+                    // shuffles, two rsqrt and a few multiplies.  Every lane updates all 16 entries
+                    // of its row: those right of its own diagonal become scratch (no other lane reads
+                    // them; the factor mode restores its zeros below).  Each lane keeps its own
+                    // pivot's values and writes them afterwards.
                     const int lb0 = lane & 16;
                     const unsigned mask = 0xFFFFu << lb0;
                     float rl_mine = 1.f, e_mine = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const float e = __shfl_sync(mask, v[c], lb0 + c);   // excess of column c
-                        const float rlc = rsqrtf(1.f + e);
-                        const float li = v[c] * rlc;                        // L_ii,c for ii > c
+                    for (int c = 0; c < 16; c += 2) {
+                        const float e0 = __shfl_sync(mask, v[c], lb0 + c);           // excess of column c
+                        const float a10 = __shfl_sync(mask, v[c], lb0 + c + 1);      // entry (c+1, c)
+                        const float e1 = __shfl_sync(mask, v[c + 1], lb0 + c + 1);   // entry (c+1, c+1)
+                        const float r0 = rsqrt_ftz(1.f + e0);                           // 1 / L_cc
+                        const float l10 = a10 * r0;                                  // L_c+1,c
+                        const float e1u = fmaf(-l10, l10, e1);                       // excess of column c+1
+                        const float r1 = rsqrt_ftz(1.f + e1u);                          // 1 / L_c+1,c+1
+                        const float li0 = v[c] * r0;                                 // L_ii,c for ii > c
+                        const float li1 = fmaf(-li0, l10, v[c + 1]) * r1;            // L_ii,c+1 for ii > c+1
+                        // v[c2] -= L_ii,c L_c2,c + L_ii,c+1 L_c2,c+1 with L_c2,c = w0 r0 and
+                        // L_c2,c+1 = (w1 - L_c2,c l10) r1, gathered per shuffled value
+                        const float g1 = li1 * r1;
+                        const float g0 = fmaf(-g1, l10, li0) * r0;
 #pragma unroll
-                        for (int c2 = 0; c2 < 16; ++c2) {
-                            if (c2 > c) {
-                                const float w = __shfl_sync(mask, v[c], lb0 + c2);
-                                const float u = fmaf(-li, w * rlc, v[c2]);
-                                v[c2] = ii >= c2 ? u : v[c2];
-                            }
+                        for (int c2 = c + 2; c2 < 16; ++c2) {
+                            const float w0 = __shfl_sync(mask, v[c], lb0 + c2);
+                            const float w1 = __shfl_sync(mask, v[c + 1], lb0 + c2);
+                            v[c2] = fmaf(-g1, w1, fmaf(-g0, w0, v[c2]));
                         }
-                        const bool piv = ii == c;
-                        v[c] = piv ? (1.f + e) * rlc : (ii > c ? li : v[c]);  // L_cc on the pivot row
-                        rl_mine = piv ? rlc : rl_mine;
-                        e_mine = piv ? e : e_mine;
+                        const bool piv0 = ii == c, piv1 = ii == c + 1;
+                        v[c] = piv0 ? (1.f + e0) * r0 : (ii > c ? li0 : v[c]);            // L_cc on its row
+                        v[c + 1] = piv1 ? (1.f + e1u) * r1 : (ii > c + 1 ? li1 : v[c + 1]);
+                        rl_mine = piv0 ? r0 : (piv1 ? r1 : rl_mine);
+                        e_mine = piv0 ? e0 : (piv1 ? e1u : e_mine);
+                    }
+                    if (FACTOR) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            if (c > ii) v[c] = 0.f;
                     }
                     s_rl[ii] = rl_mine;
                     if (!FACTOR && ii < nb && ok && dcheck(start + j0 + ii < N, st))
