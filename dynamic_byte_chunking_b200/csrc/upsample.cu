@@ -12,6 +12,7 @@
 #include "bins.cuh"
 #include "common.cuh"
 #include "tc.cuh"
+#include "tma_host.cuh"
 
 namespace dbc {
 namespace up {
@@ -101,8 +102,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(int64_t N, int nbins, Layo
 
 // Grouped GEMM on tcgen05: one CTA = 128 positions of one bin x up to 256
 // output columns.  A = the positions' chunk vectors g_c (gathered rows,
-// K-major), B = W_b (row-major [d_g][d_l], read MN-major), fp32 accumulators
-// in TMEM; the epilogue adds h_t and scatters the rows back to their positions.
+// K-major, cp.async by all threads), B = W_b (row-major [d_g][d_l], read
+// MN-major, TMA tile loads issued by one thread: tensor map over this GPU's own
+// memory, no multicast), fp32 accumulators in TMEM; the epilogue adds h_t and
+// scatters the rows back to their positions.
 struct BinTC {
     static constexpr int NS = 3;
     static constexpr uint32_t A_BYTES = 128 * 128;
@@ -115,12 +118,12 @@ struct BinTC {
 };
 
 template <class IN>
-__global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16 *__restrict__ G, int64_t dg,
-                                                             const IN *__restrict__ H, int64_t dl,
-                                                             const __nv_bfloat16 *__restrict__ W, int nbins,
+__global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
+                                                             const __nv_bfloat16 *__restrict__ G, int64_t dg,
+                                                             const IN *__restrict__ H, int64_t dl, int nbins,
                                                              Layout L, float *__restrict__ S, int64_t N, int32_t *st) {
     extern __shared__ uint8_t smraw[];
-    __shared__ uint64_t mbar[BinTC::NS];
+    __shared__ uint64_t mbar[BinTC::NS], wbar[BinTC::NS];      // stage consumed by the MMAs / W_b bytes landed
     __shared__ uint32_t tmem_base;
     __shared__ int32_t pos[128], grow[128];
     const int tile = blockIdx.x;
@@ -140,27 +143,34 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16
     const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
     if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
     if (tid == 0) {
-        for (int i = 0; i < BinTC::NS; ++i) tc::mbar_init(&mbar[i], 1);
+        for (int i = 0; i < BinTC::NS; ++i) {
+            tc::mbar_init(&mbar[i], 1);
+            tc::mbar_init(&wbar[i], 1);
+        }
         tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tmW);
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = tmem_base;
-    const __nv_bfloat16 *Wb = W + (size_t)b * dg * dl + n0;
     const int nchunks = (int)(dg / 64);
-    const int nb8 = nt / 8;
     auto load = [&](int c, uint32_t sa) {
         const uint32_t sb = sa + BinTC::A_BYTES;
-        for (int e = tid; e < 128 * 8; e += 256) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + 256 * i;
             const int r = e >> 3, ch = e & 7;
             const int g = grow[r];
             const __nv_bfloat16 *src = G + (size_t)(g >= 0 ? g : 0) * dg + c * 64 + ch * 8;
             tc::cp_async16(sa + tc::kmajor_off(r, ch * 8), src, g >= 0 ? 16u : 0u);
         }
-        for (int e = tid; e < 64 * nb8; e += 256) {
-            const int k = e / nb8, n8 = e - (e / nb8) * nb8;
-            tc::cp_async16(sb + tc::mnmajor_off(n8 * 8, k, 8192), Wb + (size_t)(c * 64 + k) * dl + n8 * 8, 16u);
+        if (tid == 0) {
+            // W_b rows c*64 .. +63, columns n0 .. n0 + nt: nt / 64 boxes of 64 x 64 (8 KB each)
+            uint64_t *bar = &wbar[c % BinTC::NS];
+            tc::mbar_arrive_expect_tx(bar, (uint32_t)(nt / 64) * 8192u);
+            for (int nq = 0; nq < nt / 64; ++nq)
+                tc::tma_load_2d(sb + (uint32_t)nq * 8192u, &tmW, bar, (int)(n0 + nq * 64), b * (int)dg + c * 64);
         }
     };
     const uint32_t idesc = tc::idesc_bf16(128, nt, false, true);
@@ -172,12 +182,15 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16
         tc::cp_async_commit();
         if (kPrefetchH && c == 0) {
             // residual rows of this tile: [128][nt] bf16, row-major (zeros for empty rows)
-            const int nc = nt / 8;
-            for (int e = tid; e < 128 * nc; e += 256) {
-                const int r = e / nc, ch = e - (e / nc) * nc;
+            const int nc = nt / 8;                               // 16-byte pieces per row, at most 32
+#pragma unroll 4
+            for (int e = tid; e < 128 * 32; e += 256) {
+                const int r = e >> 5, ch = e & 31;
                 const int p = pos[r];
-                const IN *src = H + (size_t)(p >= 0 ? p : 0) * dl + n0 + ch * 8;
-                tc::cp_async16(hbuf + (uint32_t)(r * nt + ch * 8) * 2, src, p >= 0 ? 16u : 0u);
+                if (ch < nc) {
+                    const IN *src = H + (size_t)(p >= 0 ? p : 0) * dl + n0 + ch * 8;
+                    tc::cp_async16(hbuf + (uint32_t)(r * nt + ch * 8) * 2, src, p >= 0 ? 16u : 0u);
+                }
             }
             tc::cp_async_commit();
         }
@@ -193,6 +206,7 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __nv_bfloat16
         tc::fence_async_smem();
         __syncthreads();
         if (tid == 0) {
+            ok &= tc::mbar_wait(&wbar[c % BinTC::NS], (uint32_t)(c / BinTC::NS) & 1u, st);
             tc::fence_after_sync();
             const uint32_t sa = base + (uint32_t)(c % BinTC::NS) * BinTC::STAGE, sb = sa + BinTC::A_BYTES;
 #pragma unroll
@@ -263,6 +277,10 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
                          int64_t N, int64_t d_l, const int64_t *idx, const int64_t *idx_offsets, int64_t rows,
                          const void *W_bin, int nbins, int mode, float *S, const Layout &L, int32_t *dev_status,
                          cudaStream_t s) {
+    // W_bin as one [nbins * d_g][d_l] bf16 matrix read in 64 x 64 boxes (checked before any launch)
+    if (reinterpret_cast<uintptr_t>(W_bin) & 15) return DBC_ERR_INVALID_ARG;
+    CUtensorMap tmW;
+    if (!tma::encode_bf16_rows(&tmW, W_bin, (uint64_t)nbins * (uint64_t)d_g, (uint64_t)d_l, 64)) return DBC_ERR_CUDA;
     cudaMemsetAsync(L.hist, 0, sizeof(int32_t) * kMaxBins, s);
     const int sms = num_sms();
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (int64_t)sms * 8));
@@ -274,14 +292,14 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
         cudaFuncSetAttribute(bin_gemm_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)BinTC::smem<__nv_bfloat16>());
         bin_gemm_tc_kernel<__nv_bfloat16><<<g, 256, BinTC::smem<__nv_bfloat16>(), s>>>(
-            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, N, dev_status);
+            tmW, static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l, nbins, L,
+            S, N, dev_status);
     } else {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)BinTC::smem<float>());
         bin_gemm_tc_kernel<float><<<g, 256, BinTC::smem<float>(), s>>>(
-            static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l,
-            static_cast<const __nv_bfloat16 *>(W_bin), nbins, L, S, N, dev_status);
+            tmW, static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l, nbins, L, S, N,
+            dev_status);
     }
     count_launches(4);
     return launch_status();
