@@ -228,7 +228,7 @@ struct GramTC {
 
 template <int D>
 __global__ void __launch_bounds__(256, 1) gram_tc_kernel(const __nv_bfloat16 *__restrict__ H, Segs S,
-                                                          float *aug, size_t mat_stride, int32_t *st) {
+                                                          float *aug, size_t mat_stride, bool lower, int32_t *st) {
     using C = GramTC<D>;
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[C::NS];
@@ -270,6 +270,9 @@ __global__ void __launch_bounds__(256, 1) gram_tc_kernel(const __nv_bfloat16 *__
         if (c < nchunks) load(c); else tc::cp_async_commit();
     }
     constexpr uint32_t idesc = tc::idesc_bf16(128, D < 256 ? D : 256, true, true);
+    // lower: the first 128-row block only needs its first 128 columns (D = 256 with two row blocks)
+    constexpr uint32_t idesc_half = tc::idesc_bf16(128, 128, true, true);
+    const bool half0 = lower && D == 256 && C::NMB == 2;
     for (int c = 0; c < nchunks; ++c) {
         const int cn = c + C::NS - 1;
         if (cn < nchunks) {
@@ -292,8 +295,8 @@ __global__ void __launch_bounds__(256, 1) gram_tc_kernel(const __nv_bfloat16 *__
 #pragma unroll
                     for (int nb = 0; nb < (D + 255) / 256; ++nb) {
                         const uint64_t bd = tc::sdesc(sb + (uint32_t)(4 * nb) * C::LBO + kk * 2048, C::LBO, 1024);
-                        tc::mma_bf16(tbase + (uint32_t)(m * D + nb * 256), ad, bd, idesc,
-                                     (c > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_bf16(tbase + (uint32_t)(m * D + nb * 256), ad, bd,
+                                     (half0 && m == 0) ? idesc_half : idesc, (c > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
             }
@@ -311,7 +314,8 @@ __global__ void __launch_bounds__(256, 1) gram_tc_kernel(const __nv_bfloat16 *__
         // row block each (two blocks) or one half of the columns each (one block)
         const int slot = warp >> 2, lg = warp & 3;
         const int m = C::NMB == 2 ? slot : 0;
-        const int cbeg = C::NMB == 2 ? 0 : slot * (D / 2), cend = C::NMB == 2 ? D : cbeg + D / 2;
+        const int cbeg = C::NMB == 2 ? 0 : slot * (D / 2);
+        const int cend = C::NMB == 2 ? ((half0 && m == 0) ? 128 : D) : cbeg + D / 2;
         {
             const int row = (mb0 + m) * 128 + lg * 32 + lane;
 #pragma unroll 1
@@ -562,11 +566,11 @@ __global__ void __launch_bounds__(256) first_seg_kernel(const IN *__restrict__ H
 
 template <int D>
 void launch_gram_tc(const __nv_bfloat16 *H, int64_t ns, const Segs &segs, float *mats, size_t mat_stride,
-                    int32_t *st, cudaStream_t stream) {
+                    int32_t *st, cudaStream_t stream, bool lower = false) {
     using C = GramTC<D>;
     cudaFuncSetAttribute(gram_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     gram_tc_kernel<D><<<dim3((unsigned)ns, (unsigned)C::GROUPS), 256, C::SMEM, stream>>>(H, segs, mats,
-                                                                                       mat_stride, st);
+                                                                                       mat_stride, lower, st);
 }
 
 inline void launch_gram(const float *H, int64_t d, int64_t ns, const Layout &L, int32_t *st,

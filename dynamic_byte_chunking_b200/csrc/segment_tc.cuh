@@ -61,10 +61,13 @@ inline Layout2 carve2(void *ws, int64_t rows, int64_t N, int64_t d) {
 // ---------------------------------------------------------------- prefix
 // In place over a row's segments: Gram -> P_s = c sum_{s'<s} G_s' (float64
 // running sum, fp32 store).
-__global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c, size_t stride) {
+__global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c, size_t stride,
+                                                      bool lower32 = false) {
     const int64_t r = blockIdx.x;
     const int64_t e4 = (int64_t)blockIdx.y * 256 + threadIdx.x;        // float4 index
     if (e4 * 4 >= d * d) return;
+    // lower32: the consumer reads row i only up to the end of its 32-column block
+    if (lower32 && (((4 * e4) % d) >> 5) > (((4 * e4) / d) >> 5)) return;
     const int s0 = S.row_seg0[r], s1 = S.row_seg0[r + 1];
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
     for (int sb = s0; sb < s1; sb += 16) {
@@ -503,9 +506,10 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kLmaxTmem, L.segs, st);
     const bool fused = launch_gram_prefix(H, N, rows, ns, L.segs, L.P, nullptr, c, st, stream);
     if (!fused) {
-        launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream);
+        // the factor kernel reads each row of P_s up to the end of its 32-column block only
+        launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream, true);
         prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
-            L.segs, L.P, D, c, (size_t)D * D);
+            L.segs, L.P, D, c, (size_t)D * D, true);
     }
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
