@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(1024) seg_table_kernel(const int64_t *offsets,
                                                          int32_t *st) {
     __shared__ int64_t wsum[32];
     __shared__ int64_t carry;
+    __shared__ int64_t sh_excl[1024], sh_a[1024], sh_n[1024], sh_cnt[1024];   // per row of the current block
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (tid == 0) carry = 0;
     __syncthreads();
@@ -129,15 +130,22 @@ __global__ void __launch_bounds__(1024) seg_table_kernel(const int64_t *offsets,
         }
         __syncthreads();
         const int64_t excl = carry + (wid ? wsum[wid - 1] : 0) + x - cnt;
-        if (r < rows) {
-            S.row_seg0[r] = (int32_t)excl;
-            for (int64_t k = 0; k < cnt && excl + k < ns; ++k) {
+        if (r < rows) S.row_seg0[r] = (int32_t)excl;
+        sh_excl[tid] = excl;
+        sh_a[tid] = a;
+        sh_n[tid] = n;
+        sh_cnt[tid] = cnt;
+        __syncthreads();
+        // the entries: warp w fills the rows w, w + 32, ... of this block of rows, a lane per segment
+        for (int rr = wid; rr < (int)blockDim.x && base + rr < rows; rr += (int)(blockDim.x >> 5)) {
+            const int64_t e0 = sh_excl[rr], a0 = sh_a[rr], n0 = sh_n[rr], c0 = sh_cnt[rr];
+            for (int64_t k = lane; k < c0 && e0 + k < ns; k += 32) {
                 const int64_t s0 = seg_bound(k, lmax);
-                const int64_t s1 = min(n, seg_bound(k + 1, lmax));
-                const int64_t s = excl + k;
-                S.start[s] = a + s0;
+                const int64_t s1 = min(n0, seg_bound(k + 1, lmax));
+                const int64_t s = e0 + k;
+                S.start[s] = a0 + s0;
                 S.len[s] = (int32_t)(s1 - s0);
-                S.row[s] = (int32_t)r;
+                S.row[s] = (int32_t)(base + rr);
                 S.k[s] = (int32_t)k;
             }
         }

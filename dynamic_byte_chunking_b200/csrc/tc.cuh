@@ -155,6 +155,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Zeros into 16 lanes (from the address's lane, a multiple of 16 inside the
+// warp's quarter) x 32 or 16 consecutive columns: the 16x256b shape (16 lanes
+// x 8 columns) repeated along the columns; the values are all zero, so the
+// register-to-element order of the shape does not matter.
+__device__ __forceinline__ void tmem_st_zero16x32(uint32_t taddr) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+        "r"(0u)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_zero16x16(uint32_t taddr) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(0u)
+                 : "memory");
+}
+
 // The same load without the wait: several loads may be in flight before one
 // tmem_wait_ld(); the registers must not be read before that wait.
 __device__ __forceinline__ void tmem_ld16_nw(uint32_t taddr, uint32_t (&r)[16]) {

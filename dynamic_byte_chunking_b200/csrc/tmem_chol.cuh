@@ -349,8 +349,8 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             // (committed to mbar[1]).  Panel j+1 waits for mbar[0] only, so the bulk of the update
             // runs under its factorization.  In the factor mode the rows of the diagonal block must
             // start their B entries right of the panel from zero: the other warp of their TMEM lane
-            // group resets those entries once the previous panel's bulk update has landed, while the
-            // diagonal block is being factored.
+            // group resets those entries once the previous panel's bulk update has landed, after its
+            // own solve.
             const int npan = (n + 15) / 16;
             // phase bookkeeping: panel j < npan - 1 commits once to each barrier; completion k of a
             // barrier is awaited with parity (base + k) & 1
@@ -372,39 +372,6 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 __syncwarp();
                 tc::tmem_ld16(trow + (uint32_t)j0, v);
                 const int gd = (j0 & 127) >> 5, bd = j0 >> 7;     // lane group, row block of the block rows
-                if (FACTOR && j1 < n && warp == (1 - bd) * 4 + gd) {   // warp-uniform: the reset helper
-                    bool okh = ok;
-                    if (j > 0 && okh) {
-                        okh = tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(j - 1)) & 1u, st);   // previous bulk update
-                        tc::fence_after_sync();
-                    }
-                    okh = __all_sync(0xffffffffu, okh);
-                    if (okh) {
-                        const int lrow = bd * 128 + gd * 32 + lane;   // row of this lane in those columns
-                        const bool zero = lrow >= j0 && lrow < j0 + 16;
-                        const uint32_t tb = tbase + ((uint32_t)(gd * 32) << 16) + (uint32_t)(bd * 256);
-#pragma unroll 1
-                        for (int c0 = j1; c0 < D; c0 += 32) {
-                            const int cnt = min(2, (D - c0) >> 4);      // warp-uniform
-                            uint32_t r4[2][16];
-#pragma unroll
-                            for (int q = 0; q < 2; ++q)
-                                if (q < cnt) tc::tmem_ld16_nw(tb + (uint32_t)(c0 + 16 * q), r4[q]);
-                            tc::tmem_wait_ld();
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                if (q < cnt) {
-                                    float t16[16];
-#pragma unroll
-                                    for (int i = 0; i < 16; ++i) t16[i] = zero ? 0.f : __uint_as_float(r4[q][i]);
-                                    tc::tmem_st16(tb + (uint32_t)(c0 + 16 * q), t16);
-                                }
-                            }
-                        }
-                        tc::tmem_wait_st();
-                    }
-                    ok &= okh;
-                }
                 if (FACTOR && diag) {
                     // right of its diagonal a row carries B, which only receives contributions from
                     // columns at or after its own: what earlier updates left there is dropped
@@ -414,43 +381,60 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 }
                 float a[16];
                 if (diag) {
-                    // Two pivots per step (branch-free, selects only, so the half-warp stays converged
-                    // for its shuffles): the 2 x 2 diagonal block of columns (c, c+1) is factored
-                    // from three broadcasts taken at once, and both columns are applied to the rest
-                    // of the row together, so the serial path per pivot pair is one round of
-                    // shuffles, two rsqrt and a few multiplies.  Every lane updates all 16 entries
-                    // of its row: those right of its own diagonal become scratch (no other lane reads
-                    // them; the factor mode restores its zeros below).  Each lane keeps its own
-                    // pivot's values and writes them afterwards.
+                    // Four pivots per step (branch-free, selects only, so the half-warp stays converged
+                    // for its shuffles): every lane takes the 4 x 4 diagonal block of columns c .. c+3
+                    // (ten broadcasts at once) and factors it itself, solves its own row's four values
+                    // against it (l = L4^-1 x) and applies the four columns to the rest of its row as
+                    // v -= g . w with g = L4^-T l and w the four values of the other row, so the serial
+                    // path per four pivots is one round of shuffles, four rsqrt and a few fma.  Every
+                    // lane updates all 16 entries of its row: those right of its own diagonal become
+                    // scratch (no other lane reads them; the factor mode restores its zeros below).
+                    // Each lane keeps its own pivot's values and writes them afterwards.
                     const int lb0 = lane & 16;
                     const unsigned mask = 0xFFFFu << lb0;
                     float rl_mine = 1.f, e_mine = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 16; c += 2) {
-                        const float e0 = __shfl_sync(mask, v[c], lb0 + c);           // excess of column c
-                        const float a10 = __shfl_sync(mask, v[c], lb0 + c + 1);      // entry (c+1, c)
-                        const float e1 = __shfl_sync(mask, v[c + 1], lb0 + c + 1);   // entry (c+1, c+1)
-                        const float r0 = rsqrt_ftz(1.f + e0);                           // 1 / L_cc
-                        const float l10 = a10 * r0;                                  // L_c+1,c
-                        const float e1u = fmaf(-l10, l10, e1);                       // excess of column c+1
-                        const float r1 = rsqrt_ftz(1.f + e1u);                          // 1 / L_c+1,c+1
-                        const float li0 = v[c] * r0;                                 // L_ii,c for ii > c
-                        const float li1 = fmaf(-li0, l10, v[c + 1]) * r1;            // L_ii,c+1 for ii > c+1
-                        // v[c2] -= L_ii,c L_c2,c + L_ii,c+1 L_c2,c+1 with L_c2,c = w0 r0 and
-                        // L_c2,c+1 = (w1 - L_c2,c l10) r1, gathered per shuffled value
-                        const float g1 = li1 * r1;
-                        const float g0 = fmaf(-g1, l10, li0) * r0;
+                    for (int c = 0; c < 16; c += 4) {
+                        float a[4][4];                                       // a[p][q], q <= p
 #pragma unroll
-                        for (int c2 = c + 2; c2 < 16; ++c2) {
+                        for (int p = 0; p < 4; ++p)
+#pragma unroll
+                            for (int q = 0; q <= p; ++q) a[p][q] = __shfl_sync(mask, v[c + q], lb0 + c + p);
+                        // L4 (unit-free: the diagonal of I + a is 1 + e)
+                        const float r0 = rsqrt_ftz(1.f + a[0][0]);
+                        const float L10 = a[1][0] * r0, L20 = a[2][0] * r0, L30 = a[3][0] * r0;
+                        const float e1 = fmaf(-L10, L10, a[1][1]);
+                        const float r1 = rsqrt_ftz(1.f + e1);
+                        const float L21 = fmaf(-L20, L10, a[2][1]) * r1, L31 = fmaf(-L30, L10, a[3][1]) * r1;
+                        const float e2 = fmaf(-L21, L21, fmaf(-L20, L20, a[2][2]));
+                        const float r2 = rsqrt_ftz(1.f + e2);
+                        const float L32 = fmaf(-L31, L21, fmaf(-L30, L20, a[3][2])) * r2;
+                        const float e3 = fmaf(-L32, L32, fmaf(-L31, L31, fmaf(-L30, L30, a[3][3])));
+                        const float r3 = rsqrt_ftz(1.f + e3);
+                        // this row's factor entries in the four columns
+                        const float l0 = v[c] * r0;
+                        const float l1 = fmaf(-l0, L10, v[c + 1]) * r1;
+                        const float l2 = fmaf(-l1, L21, fmaf(-l0, L20, v[c + 2])) * r2;
+                        const float l3 = fmaf(-l2, L32, fmaf(-l1, L31, fmaf(-l0, L30, v[c + 3]))) * r3;
+                        const float g3 = l3 * r3;
+                        const float g2 = fmaf(-g3, L32, l2) * r2;
+                        const float g1 = fmaf(-g3, L31, fmaf(-g2, L21, l1)) * r1;
+                        const float g0 = fmaf(-g3, L30, fmaf(-g2, L20, fmaf(-g1, L10, l0))) * r0;
+#pragma unroll
+                        for (int c2 = c + 4; c2 < 16; ++c2) {
                             const float w0 = __shfl_sync(mask, v[c], lb0 + c2);
                             const float w1 = __shfl_sync(mask, v[c + 1], lb0 + c2);
-                            v[c2] = fmaf(-g1, w1, fmaf(-g0, w0, v[c2]));
+                            const float w2 = __shfl_sync(mask, v[c + 2], lb0 + c2);
+                            const float w3 = __shfl_sync(mask, v[c + 3], lb0 + c2);
+                            v[c2] = fmaf(-g3, w3, fmaf(-g2, w2, fmaf(-g1, w1, fmaf(-g0, w0, v[c2]))));
                         }
-                        const bool piv0 = ii == c, piv1 = ii == c + 1;
-                        v[c] = piv0 ? (1.f + e0) * r0 : (ii > c ? li0 : v[c]);            // L_cc on its row
-                        v[c + 1] = piv1 ? (1.f + e1u) * r1 : (ii > c + 1 ? li1 : v[c + 1]);
-                        rl_mine = piv0 ? r0 : (piv1 ? r1 : rl_mine);
-                        e_mine = piv0 ? e0 : (piv1 ? e1u : e_mine);
+                        const float e0 = a[0][0];
+                        v[c] = ii == c ? (1.f + e0) * r0 : l0;                  // L_cc on its row
+                        v[c + 1] = ii == c + 1 ? (1.f + e1) * r1 : l1;
+                        v[c + 2] = ii == c + 2 ? (1.f + e2) * r2 : l2;
+                        v[c + 3] = ii == c + 3 ? (1.f + e3) * r3 : l3;
+                        rl_mine = ii == c ? r0 : (ii == c + 1 ? r1 : (ii == c + 2 ? r2 : (ii == c + 3 ? r3 : rl_mine)));
+                        e_mine = ii == c ? e0 : (ii == c + 1 ? e1 : (ii == c + 2 ? e2 : (ii == c + 3 ? e3 : e_mine)));
                     }
                     if (FACTOR) {
 #pragma unroll
@@ -497,6 +481,28 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 } else {
 #pragma unroll
                     for (int m = 0; m < 16; ++m) a[m] = 0.f;
+                }
+                if (FACTOR && j1 < n && warp == (1 - bd) * 4 + gd) {
+                    // the reset helper, the other warp of the block rows' TMEM lane quarter: right of the
+                    // panel the block rows carry B, which restarts from zero once the previous panel's
+                    // bulk update has landed (done here, after the solve, so that its wait is hidden;
+                    // this panel's updates of those entries are issued after the next vote).  Stores of
+                    // zeros to those 16 lanes only, nothing read back.
+                    bool okh = ok;
+                    if (j > 0 && okh) {
+                        okh = tc::mbar_wait(&mbar[1], (base1 + (uint32_t)(j - 1)) & 1u, st);   // previous bulk update
+                        tc::fence_after_sync();
+                    }
+                    okh = __all_sync(0xffffffffu, okh);
+                    if (okh) {
+                        const uint32_t tz = tbase + ((uint32_t)(gd * 32 + (j0 & 31)) << 16) + (uint32_t)(bd * 256);
+                        int c0 = j1;
+#pragma unroll 1
+                        for (; c0 + 32 <= D; c0 += 32) tc::tmem_st_zero16x32(tz + (uint32_t)c0);
+                        if (c0 < D) tc::tmem_st_zero16x16(tz + (uint32_t)c0);
+                        tc::tmem_wait_st();
+                    }
+                    ok &= okh;
                 }
                 if (FACTOR) {
                     // the panel's final values stay in TMEM (B right of the diagonal, zero left of it
