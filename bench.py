@@ -52,9 +52,9 @@ def parse():
     ap.add_argument("--families", default="tiny,byteflow,bytegen,wide,ragged",
                     help="workload families measured by --rows (comma-separated)")
     ap.add_argument("--probe", default=None, metavar="FAMILY",
-                    help="run the path twice on one workload family (coding rate, Top-K, gather, upsample, and the "
-                         "router with EMA where the family has router weights), check the device status and exit: "
-                         "a short, fixed launch sequence for profilers")
+                    help="run the path twice on one workload family (coding rate, Top-K, gather, upsample, the "
+                         "router with EMA where the family has router weights, the Canon layer for bf16 "
+                         "families), check the device status and exit: a short, fixed launch sequence for profilers")
     ap.add_argument("--traffic-from", default=None, metavar="CSV",
                     help="convert an ncu --csv launch list with dram__bytes_read.sum and dram__bytes_write.sum "
                          "(taken on this workload) into profiles/dram_traffic_byteflow.json, then exit")
@@ -488,6 +488,13 @@ def run_probe(family, reps=2):
           if w.W_bin is not None and w.W_proj is None else None)
     Wq = torch.from_numpy(w.Wq.view(np.int16)).view(torch.bfloat16).to(dev) if w.Wq is not None else None
     Wk = torch.from_numpy(w.Wk.view(np.int16)).view(torch.bfloat16).to(dev) if w.Wk is not None else None
+    canon = None
+    if w.dtype == "bf16":
+        gen = np.random.default_rng(11)
+        to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        canon = (to_dev(workloads.bf16_bits((gen.standard_normal((d, 4)) * 0.5).astype(np.float32))),
+                 to_dev(workloads.bf16_bits((gen.standard_normal(d) * 0.02).astype(np.float32))),
+                 torch.empty(N, d, dtype=torch.bfloat16, device=dev))
     for _ in range(reps):
         dbc.chunk_coding_rate(Hx, w.eps2, offsets=o, T=T, dR=dR, workspace=ws, dev_status=st)
         idx, io = dbc.chunk_topk_select(dR, Kt, rows=rows, T=T, offsets=o, total=total, dev_status=st)
@@ -496,6 +503,8 @@ def run_probe(family, reps=2):
             dbc.chunk_upsample(Z, H, idx, io, Wb, rows=rows, T=T, offsets=o, dev_status=st)
         if Wq is not None:
             dbc.hnet_route(Hx, Wq, Wk, offsets=o, T=T, do_ema=True, dev_status=st)
+        if canon is not None:
+            dbc.canon_conv1d(Hx, canon[0], canon[1], offsets=o, T=T, residual=True, out=canon[2], dev_status=st)
     torch.cuda.synchronize()
     if st.item() != 0:
         raise RuntimeError(f"device status flags {st.item():#x}")
