@@ -61,13 +61,27 @@ inline Layout2 carve2(void *ws, int64_t rows, int64_t N, int64_t d) {
 // ---------------------------------------------------------------- prefix
 // In place over a row's segments: Gram -> P_s = c sum_{s'<s} G_s' (float64
 // running sum, fp32 store).
+// Number of float4 entries of a d x d matrix left of the end of each row's 32-column block.
+__host__ __device__ __forceinline__ int64_t lower32_count(int64_t d) {
+    const int64_t nb = d / 32;
+    return 128 * nb * (nb + 1);
+}
+
 __global__ void __launch_bounds__(256) prefix2_kernel(Segs S, float *aug2, int64_t d, double c, size_t stride,
                                                       bool lower32 = false) {
     const int64_t r = blockIdx.x;
-    const int64_t e4 = (int64_t)blockIdx.y * 256 + threadIdx.x;        // float4 index
+    int64_t e4 = (int64_t)blockIdx.y * 256 + threadIdx.x;              // float4 index
+    if (lower32) {
+        // the consumer reads row i only up to the end of its 32-column block: threads cover those
+        // entries only, row block rb (32 rows of 8 (rb + 1) float4 each) after the ones above it
+        if (e4 >= lower32_count(d)) return;
+        int rb = 0;
+        while (128 * (int64_t)(rb + 1) * (rb + 2) <= e4) ++rb;
+        const int64_t local = e4 - 128 * (int64_t)rb * (rb + 1);
+        const int64_t w = 8 * (int64_t)(rb + 1);
+        e4 = (rb * 32 + local / w) * (d / 4) + local % w;
+    }
     if (e4 * 4 >= d * d) return;
-    // lower32: the consumer reads row i only up to the end of its 32-column block
-    if (lower32 && (((4 * e4) % d) >> 5) > (((4 * e4) / d) >> 5)) return;
     const int s0 = S.row_seg0[r], s1 = S.row_seg0[r + 1];
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
     for (int sb = s0; sb < s1; sb += 16) {
@@ -508,7 +522,7 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     if (!fused) {
         // the factor kernel reads each row of P_s up to the end of its 32-column block only
         launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream, true);
-        prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
+        prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((lower32_count(D) + 255) / 256)), 256, 0, stream>>>(
             L.segs, L.P, D, c, (size_t)D * D, true);
     }
     const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);

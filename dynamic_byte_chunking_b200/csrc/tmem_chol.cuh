@@ -190,17 +190,18 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             // ---------------- load the matrix into TMEM
             if (FACTOR) {
                 // each thread moves its own row of the c-scaled prefix Gram into TMEM: the lower
-                // triangle (loaded straight from global memory, 8 loads in flight) and zeros right
-                // of it, where B = L^{-T} accumulates
+                // triangle (loaded straight from global memory, 32-column chunks double-buffered in
+                // registers so that two chunks' loads are in flight) and zeros right of it, where
+                // B = L^{-T} accumulates
                 const float *P = Pbuf + (size_t)s * D * D + (size_t)row * D;
-#pragma unroll 1
-                for (int q = 0; q < D / 32; ++q) {
-                    float4 x[8];
-                    const bool any = q * 32 <= row;                      // warp-uniform
-                    if (any) {
+                auto ldq = [&](int q, float4 (&x)[8]) {
+                    if (q * 32 <= row) {                                 // warp-uniform
 #pragma unroll
                         for (int i = 0; i < 8; ++i) x[i] = *reinterpret_cast<const float4 *>(P + q * 32 + 4 * i);
                     }
+                };
+                auto stq = [&](int q, const float4 (&x)[8]) {
+                    const bool any = q * 32 <= row;
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         float v[16];
@@ -213,6 +214,17 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                         }
                         tc::tmem_st16(trow + (uint32_t)(q * 32 + j * 16), v);
                     }
+                };
+                float4 xa[8], xb[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) xa[i] = xb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                ldq(0, xa);
+#pragma unroll 1
+                for (int q = 0; q < D / 32; q += 2) {
+                    ldq(q + 1, xb);
+                    stq(q, xa);
+                    if (q + 2 < D / 32) ldq(q + 2, xa);
+                    stq(q + 1, xb);
                 }
                 tc::tmem_wait_st();
             } else {
