@@ -282,7 +282,6 @@ constexpr int kCThreads = 256;
 constexpr int kCWarps = kCThreads / 32;
 constexpr int kSliceKeys = 8192;                       // keys per CTA slice (32 KB)
 constexpr int kClusterKeys = kCluster * kSliceKeys;    // candidates per row on this path
-constexpr int kWarpKeys = kSliceKeys / kCWarps;       // keys of a slice per warp (1024)
 
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     select_cluster_kernel(const float *__restrict__ dR, const int64_t *offsets, int64_t rows, int64_t T,
@@ -294,7 +293,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     __shared__ uint32_t s_bin;
     __shared__ int s_rem;
     __shared__ int s_cnt[2];                           // this slice's equal-key and selected counts
-    __shared__ int s_weq[kCWarps], s_wsel[kCWarps];    // per-warp counts, then their exclusive prefix
+    __shared__ int s_weq[kCWarps], s_wgt[kCWarps];     // per-warp equal and above counts
     cg::cluster_group cluster = cg::this_cluster();
     const int q = (int)cluster.block_rank();
     const int64_t r = blockIdx.x / kCluster;
@@ -329,7 +328,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     const int mine = max(0, k1 - k0);
     const float *row = dR + a + 1;
     bool bad = false;
-    for (int j = tid; j < mine; j += kCThreads) {
+#pragma unroll 4
+    for (int j = tid; j < mine; j += kCThreads) {     // four loads in flight
         const float f = row[k0 + j];
         bad |= !isfinite(f);
         keys[j] = key_of(f);
@@ -384,16 +384,19 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
         mask |= 255u << shift;
         rem = s_rem;
     }
-    // ordered compaction: key > v, or key == v among the first `rem` equal keys of the row.  Warp w
-    // owns keys [w * kWarpKeys, (w + 1) * kWarpKeys) of the slice and walks them 32 at a time (lane l
-    // takes key step * 32 + l: conflict-free shared loads), ranking with ballots; warps are offset by
-    // the warps before them, slices by the slices before them.
+    // ordered compaction: key > v, or key == v among the first `rem` equal keys of the row.  The
+    // slice's keys are split into eight contiguous ranges, one per warp, of a multiple of 32 keys;
+    // warp w walks its range 32 at a time (lane l takes key step * 32 + l: conflict-free shared
+    // loads), ranking with ballots; warps are offset by the warps before them, slices by the slices
+    // before them.
     const uint32_t v = prefix;
     const int lane = tid & 31, wid = tid >> 5;
     const unsigned lt = (1u << lane) - 1u;
-    const int wk0 = wid * kWarpKeys;
+    const int wkeys = ((mine + kCWarps * 32 - 1) / (kCWarps * 32)) * 32;   // keys per warp
+    const int wk0 = wid * wkeys;
+    const int wsteps = wkeys / 32;
     int n_eq = 0, n_gt = 0;                            // warp totals (every lane holds them)
-    for (int step = 0; step < kWarpKeys / 32; ++step) {
+    for (int step = 0; step < wsteps; ++step) {
         const int j = wk0 + step * 32 + lane;
         const uint32_t k = j < mine ? keys[j] : 0u;
         n_eq += __popc(__ballot_sync(0xffffffffu, j < mine && k == v));
@@ -401,31 +404,40 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     }
     if (lane == 0) {
         s_weq[wid] = n_eq;
+        s_wgt[wid] = n_gt;
     }
     __syncthreads();
     if (tid == 0) {
-        int c = 0;
-        for (int w = 0; w < kCWarps; ++w) { const int x = s_weq[w]; s_weq[w] = c; c += x; }
-        s_cnt[0] = c;                                  // equal keys of the slice
+        int e = 0, g = 0;
+        for (int w = 0; w < kCWarps; ++w) { e += s_weq[w]; g += s_wgt[w]; }
+        s_cnt[0] = e;                                  // equal keys of the slice
+        s_cnt[1] = g;                                  // keys above v in the slice
     }
     cluster.sync();
-    int eq_before = s_weq[wid];
-    for (int c = 0; c < q; ++c) eq_before += cluster.map_shared_rank(s_cnt, c)[0];
+    // One exchange gives every offset: slice c takes min(eq_c, rem - (equal keys before it)) of its
+    // equal keys, so the selected keys before this warp follow from the (equal, above) counts of
+    // the slices and warps before it.
+    int eq_before = 0, sel_before = 0;
+    for (int c = 0; c < q; ++c) {
+        const int *rc = cluster.map_shared_rank(s_cnt, c);
+        const int e = rc[0], g = rc[1];
+        const int l = rem - eq_before;
+        sel_before += g + (l <= 0 ? 0 : (l >= e ? e : l));
+        eq_before += e;
+    }
+    // this CTA's reads of the other slices' counts are done; its own may still be read
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    for (int w = 0; w < wid; ++w) {
+        const int e = s_weq[w], g = s_wgt[w];
+        const int l = rem - eq_before;
+        sel_before += g + (l <= 0 ? 0 : (l >= e ? e : l));
+        eq_before += e;
+    }
     const int left = rem - eq_before;
     const int take_eq = left <= 0 ? 0 : (left >= n_eq ? n_eq : left);
-    if (lane == 0) s_wsel[wid] = n_gt + take_eq;
-    __syncthreads();
-    if (tid == 0) {
-        int c = 0;
-        for (int w = 0; w < kCWarps; ++w) { const int x = s_wsel[w]; s_wsel[w] = c; c += x; }
-        s_cnt[1] = c;                                  // selected keys of the slice
-    }
-    cluster.sync();
-    int sel_before = s_wsel[wid];
-    for (int c = 0; c < q; ++c) sel_before += cluster.map_shared_rank(s_cnt, c)[1];
     int64_t o = 1 + (int64_t)sel_before;
     int eq_run = 0;
-    for (int step = 0; step < kWarpKeys / 32; ++step) {
+    for (int step = 0; step < wsteps; ++step) {
         const int j = wk0 + step * 32 + lane;
         const uint32_t k = j < mine ? keys[j] : 0u;
         const bool eq = j < mine && k == v;
@@ -439,7 +451,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
         o += __popc(sm);
         eq_run += __popc(em);
     }
-    cluster.sync();                                    // no CTA leaves while its counts may still be read
+    // no CTA leaves while its counts may still be read
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 }  // namespace tk
