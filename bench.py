@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="dbc", choices=["dbc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the device steps with eager launches instead of CUDA-graph replays")
     ap.add_argument("--rows", action="store_true",
                     help="time every hot-path row on its own workload family (one JSON line per row)")
     ap.add_argument("--reps", type=int, default=10)
@@ -595,6 +597,47 @@ def main():
     torch.cuda.synchronize()
     check_status("during warm-up")
 
+    # The timed steps replay each call as a CUDA graph (captured once, after the warm-up): the same
+    # kernels with the same arguments, minus the host launch gaps between them.  `gpu_launches`
+    # counts the kernels the graphs hold times the replays.
+    graphs, per_step_launches, launch_mode = None, None, "eager"
+    if not args.no_graph:
+        try:
+            calls = [
+                lambda: dbc.chunk_coding_rate(H, w.eps2, dR=dR, workspace=ws_cr, dev_status=st),
+                lambda: dbc.chunk_topk_select(dR, K, rows=rows, T=T, idx=idx, idx_offsets=io, dev_status=st),
+                lambda: dbc.chunk_gather(H, idx, io, rows=rows, T=T, total=rows * K, Z=Z, dev_status=st),
+                lambda: dbc.chunk_upsample(Z, H, idx, io, Wb, rows=rows, T=T, S=S, workspace=ws_up, dev_status=st)]
+            l0 = dbc.launch_count()
+            graphs = []
+            for c in calls:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    c()
+                graphs.append(g)
+            per_step_launches = dbc.launch_count() - l0
+            torch.cuda.synchronize()
+            for _ in range(2):
+                flush.zero_()
+                for g in graphs:
+                    g.replay()
+            torch.cuda.synchronize()
+            check_status("during the graph warm-up")
+            launch_mode = "cuda_graph"
+        except Exception as exc:          # keep the eager steps if a capture is refused
+            graphs = None
+            launch_mode = "eager (graph capture failed: %s)" % str(exc).splitlines()[0][:120]
+            torch.cuda.synchronize()
+
+    def timed_step(ev):
+        if graphs is None:
+            step(H, ev)
+            return
+        for s_, g in enumerate(graphs):
+            ev[s_].record(stream)
+            g.replay()
+        ev[4].record(stream)
+
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     gpu_id = str(local)
     try:
@@ -612,9 +655,9 @@ def main():
     launches0 = dbc.launch_count()
     for k in range(args.steps):
         flush.zero_()
-        step(H, evs[k])
+        timed_step(evs[k])
     torch.cuda.synchronize()
-    launches = dbc.launch_count() - launches0
+    launches = dbc.launch_count() - launches0 if graphs is None else per_step_launches * args.steps
     if pg:
         pg.barrier()
     time.sleep(0.2)
@@ -728,7 +771,7 @@ def main():
                            "global_batch": 8 * world,
                            "parallelism": f"dp{world}: rows of one global batch split by sharding.partition_rows",
                            "l2": "flushed by a 256 MB write before every timed step",
-                           "step": " -> ".join(stages)},
+                           "step": " -> ".join(stages), "launch": launch_mode},
                 "stage_ms": {s: float(a) for s, a in zip(stages, avg)},
                 "value_chunk": {"value": value_chunk, "unit": UNIT, "ms": t_chunk,
                                 "definition": "positions / (chunk_coding_rate + chunk_topk_select + chunk_gather)"},
