@@ -25,8 +25,6 @@ struct Layout {
     int32_t *perm;       // [N] positions grouped by bin
     int32_t *hist;       // [kMaxBins]
     int32_t *cursor;     // [kMaxBins]
-    int32_t *bin_start;  // [kMaxBins + 1]
-    int32_t *tile_start; // [kMaxBins + 1]
     size_t bytes;
 };
 
@@ -38,8 +36,6 @@ inline Layout carve(void *ws, int64_t N) {
     L.perm = c.take<int32_t>(N + 1);
     L.hist = c.take<int32_t>(kMaxBins);
     L.cursor = c.take<int32_t>(kMaxBins);
-    L.bin_start = c.take<int32_t>(kMaxBins + 1);
-    L.tile_start = c.take<int32_t>(kMaxBins + 1);
     L.bytes = c.off;
     return L;
 }
@@ -51,37 +47,53 @@ __global__ void __launch_bounds__(256) classify_kernel(const int64_t *offsets, i
     __shared__ int32_t h[kMaxBins];
     for (int b = threadIdx.x; b < nbins; b += blockDim.x) h[b] = 0;
     __syncthreads();
-    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < N;
-         p += (int64_t)gridDim.x * blockDim.x) {
-        const PosClass pc = classify_position(p, offsets, T, idx, idx_offsets, rows, nbins, mode, st);
-        L.chunk[p] = pc.chunk;
-        L.bin[p] = (uint8_t)pc.bin;
-        atomicAdd(&h[pc.bin], 1);
+    // a warp classifies 32 consecutive positions together; one shared atomic per distinct bin
+    const int lane = threadIdx.x & 31;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < N; base += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t p0 = base + (threadIdx.x & ~31);
+        if (p0 >= N) continue;                                   // warp-uniform
+        const PosClass pc = classify_warp(p0, N, offsets, T, idx, idx_offsets, rows, nbins, mode, st);
+        const int64_t p = p0 + lane;
+        const bool live = p < N;
+        if (live) {
+            L.chunk[p] = pc.chunk;
+            L.bin[p] = (uint8_t)pc.bin;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, live ? pc.bin : -1);
+        if (live && lane == __ffs(peers) - 1) atomicAdd(&h[pc.bin], __popc(peers));
     }
     __syncthreads();
     for (int b = threadIdx.x; b < nbins; b += blockDim.x)
         if (h[b]) atomicAdd(&L.hist[b], h[b]);
 }
 
-__global__ void scan_bins_kernel(int nbins, Layout L) {
-    if (threadIdx.x == 0) {
-        int32_t s = 0, t = 0;
-        for (int b = 0; b < nbins; ++b) {
-            L.bin_start[b] = s;
-            L.tile_start[b] = t;
-            L.cursor[b] = 0;
-            s += L.hist[b];
-            t += (L.hist[b] + 127) / 128;
-        }
-        L.bin_start[nbins] = s;
-        L.tile_start[nbins] = t;
+// Bin tables from the bin counts, computed by one warp of each CTA that needs them (at most 64
+// bins): bs[b] = first permutation slot of bin b, ts[b] = first 128-slot tile of bin b, each with
+// the total at index nbins.
+__device__ __forceinline__ void bin_tables(const int32_t *__restrict__ hist, int nbins, int32_t *bs, int32_t *ts) {
+    const int lane = threadIdx.x & 31;
+    const int b0 = 2 * lane, b1 = 2 * lane + 1;
+    const int32_t h0 = b0 < nbins ? hist[b0] : 0, h1 = b1 < nbins ? hist[b1] : 0;
+    const int32_t t0 = (h0 + 127) / 128, t1 = (h1 + 127) / 128;
+    int32_t hs = h0 + h1, tsum = t0 + t1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, hs, o), z = __shfl_up_sync(0xffffffffu, tsum, o);
+        if (lane >= o) { hs += y; tsum += z; }
     }
+    const int32_t he = hs - h0 - h1, te = tsum - t0 - t1;     // exclusive
+    if (b0 < nbins) { bs[b0] = he; ts[b0] = te; }
+    if (b1 < nbins) { bs[b1] = he + h0; ts[b1] = te + t0; }
+    if (lane == 31) { bs[nbins] = hs; ts[nbins] = tsum; }      // the totals (bins past nbins count 0)
 }
 
 // Positions -> their bin's slice of the permutation.  Slots are reserved per
 // block (one global atomic per bin and block), then handed out in shared memory.
 __global__ void __launch_bounds__(256) scatter_kernel(int64_t N, int nbins, Layout L) {
     __shared__ int32_t cnt[kMaxBins], base[kMaxBins];
+    __shared__ int32_t s_bs[kMaxBins + 1], s_ts[kMaxBins + 1];
+    if (threadIdx.x < 32) bin_tables(L.hist, nbins, s_bs, s_ts);
+    __syncthreads();
     for (int64_t p0 = (int64_t)blockIdx.x * blockDim.x; p0 < N; p0 += (int64_t)gridDim.x * blockDim.x) {
         for (int b = threadIdx.x; b < nbins; b += blockDim.x) cnt[b] = 0;
         __syncthreads();
@@ -95,7 +107,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(int64_t N, int nbins, Layo
         for (int q = threadIdx.x; q < nbins; q += blockDim.x)
             base[q] = cnt[q] ? atomicAdd(&L.cursor[q], cnt[q]) : 0;
         __syncthreads();
-        if (b >= 0) L.perm[L.bin_start[b] + base[b] + slot] = (int32_t)p;
+        if (b >= 0) L.perm[s_bs[b] + base[b] + slot] = (int32_t)p;
         __syncthreads();
     }
 }
@@ -126,12 +138,15 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_consta
     __shared__ uint64_t mbar[BinTC::NS], wbar[BinTC::NS];      // stage consumed by the MMAs / W_b bytes landed
     __shared__ uint32_t tmem_base;
     __shared__ int32_t pos[128], grow[128];
+    __shared__ int32_t s_bs[kMaxBins + 1], s_ts[kMaxBins + 1];
+    if (threadIdx.x < 32) bin_tables(L.hist, nbins, s_bs, s_ts);
+    __syncthreads();
     const int tile = blockIdx.x;
-    if (tile >= L.tile_start[nbins]) return;
+    if (tile >= s_ts[nbins]) return;
     int b = 0;
-    while (b + 1 < nbins && L.tile_start[b + 1] <= tile) ++b;
-    const int r0 = L.bin_start[b] + (tile - L.tile_start[b]) * 128;
-    const int cnt = min(128, L.bin_start[b + 1] - r0);
+    while (b + 1 < nbins && s_ts[b + 1] <= tile) ++b;
+    const int r0 = s_bs[b] + (tile - s_ts[b]) * 128;
+    const int cnt = min(128, s_bs[b + 1] - r0);
     const int64_t n0 = (int64_t)blockIdx.y * 256;
     const int nt = (int)(dl - n0 < 256 ? dl - n0 : 256);      // multiple of 64
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -281,11 +296,12 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
     if (reinterpret_cast<uintptr_t>(W_bin) & 15) return DBC_ERR_INVALID_ARG;
     CUtensorMap tmW;
     if (!tma::encode_bf16_rows(&tmW, W_bin, (uint64_t)nbins * (uint64_t)d_g, (uint64_t)d_l, 64)) return DBC_ERR_CUDA;
-    cudaMemsetAsync(L.hist, 0, sizeof(int32_t) * kMaxBins, s);
+    // the bin counts and the scatter cursors start at zero (adjacent in the workspace)
+    cudaMemsetAsync(L.hist, 0, (size_t)(reinterpret_cast<char *>(L.cursor + kMaxBins) - reinterpret_cast<char *>(L.hist)),
+                    s);
     const int sms = num_sms();
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((N + 255) / 256, (int64_t)sms * 8));
     classify_kernel<<<grid, 256, 0, s>>>(offsets, T, N, idx, idx_offsets, rows, nbins, mode, L, dev_status);
-    scan_bins_kernel<<<1, 32, 0, s>>>(nbins, L);
     scatter_kernel<<<grid, 256, 0, s>>>(N, nbins, L);
     dim3 g((unsigned)((N + 127) / 128 + nbins), (unsigned)((d_l + 255) / 256));
     if (dtype == DBC_BF16) {
@@ -301,7 +317,7 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
             tmW, static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l, nbins, L, S, N,
             dev_status);
     }
-    count_launches(4);
+    count_launches(3);
     return launch_status();
 }
 
