@@ -485,6 +485,7 @@ inline Layout3 carve3(void *ws, int64_t rows, int64_t N, int64_t d, int64_t ns_g
 
 #include "tmem_chol.cuh"
 #include "gram_prefix.cuh"
+#include "gram_tma.cuh"
 #include "tma_host.cuh"
 
 namespace dbc {
@@ -521,7 +522,14 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
     const bool fused = launch_gram_prefix(H, N, rows, ns, L.segs, L.P, nullptr, c, st, stream);
     if (!fused) {
         // the factor kernel reads each row of P_s up to the end of its 32-column block only
-        launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream, true);
+        CUtensorMap tmH, tmG;
+        if (tma::encode_bf16_rows(&tmH, H, (uint64_t)N, D, 64) &&
+            tma::encode_f32_rows(&tmG, L.P, (uint64_t)ns * D, D, 128)) {
+            cudaFuncSetAttribute(gram_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GramTma::SMEM);
+            gram_tma_kernel<<<(unsigned)ns, 256, GramTma::SMEM, stream>>>(tmH, tmG, L.segs, st);
+        } else {
+            launch_gram_tc<D>(H, ns, L.segs, L.P, (size_t)D * D, st, stream, true);
+        }
         prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((lower32_count(D) + 255) / 256)), 256, 0, stream>>>(
             L.segs, L.P, D, c, (size_t)D * D, true);
     }
