@@ -10,7 +10,8 @@ Metric: sequence bytes per second (byte positions of the batch / step time).
 Timing: W untimed warm-up steps, then exactly K steps, each preceded (outside
 its timed interval) by a 256 MB write that flushes the 126 MB L2; CUDA events
 on the launching stream; barrier + synchronize around the timed loop; max over
-ranks.  Under torchrun one global batch of 8 rows per rank is drawn and its
+ranks.  The timed steps replay each of the four calls as a CUDA graph captured
+after the warm-up (``--no-graph``: eager launches).  Under torchrun one global batch of 8 rows per rank is drawn and its
 rows are split over the ranks by the library's row partition (weak scaling, no
 collective on the data path).
 
