@@ -512,12 +512,29 @@ inline bool launch_gram_prefix(const __nv_bfloat16 *H, int64_t N, int64_t rows, 
     return true;
 }
 
+// The factor and in-segment Cholesky launches of ns segments (tensor maps over P and B's pieces for the
+// factor mode's TMA loads and stores).  False (nothing launched) when a tensor map cannot be encoded.
+inline bool launch_tmem_chol(const __nv_bfloat16 *H, int64_t N, int64_t ns, const Layout3 &L, float c, float *dR,
+                             int32_t *st, cudaStream_t stream) {
+    constexpr int D = 256;
+    CUtensorMap tmP, tmB;
+    if (!tma::encode_f32_rows(&tmP, L.P, (uint64_t)ns * D, D, 32)) return false;
+    if (!tma::encode_bf16_rows(&tmB, L.Bscr, (uint64_t)ns * 3 * D, D, 64)) return false;
+    const int grid = (int)std::min<int64_t>(ns, (int64_t)num_sms());
+    cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
+    cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(tmP, tmB, L.segs, L.P, L.Bscr, nullptr, N, c,
+                                                                         dR, st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(tmP, tmB, L.segs, nullptr, L.Bscr, H, N, c,
+                                                                          dR, st);
+    return true;
+}
+
 inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64_t rows, int64_t T, int64_t N,
                            float eps2, float *dR, const Layout3 &L, int32_t *st, cudaStream_t stream) {
     constexpr int D = 256;
     const double c = (double)D / (double)eps2;
     const int64_t ns = nseg_upper(rows, N, kLmaxTmem);
-    const int sms = num_sms();
     seg_table_kernel<<<1, 1024, 0, stream>>>(offsets, rows, T, N, ns, kLmaxTmem, L.segs, st);
     const bool fused = launch_gram_prefix(H, N, rows, ns, L.segs, L.P, nullptr, c, st, stream);
     if (!fused) {
@@ -533,13 +550,7 @@ inline dbc_status run_tmem(const __nv_bfloat16 *H, const int64_t *offsets, int64
         prefix2_kernel<<<dim3((unsigned)rows, (unsigned)((lower32_count(D) + 255) / 256)), 256, 0, stream>>>(
             L.segs, L.P, D, c, (size_t)D * D, true);
     }
-    const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
-    cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, (float)c,
-                                                                         dR, st);
-    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, L.Bscr, H, N, (float)c, dR,
-                                                                          st);
+    if (!launch_tmem_chol(H, N, ns, L, (float)c, dR, st, stream)) return DBC_ERR_CUDA;
     count_launches(fused ? 4 : 5);
     return launch_status();
 }
@@ -630,13 +641,7 @@ inline dbc_status run_tmem_stream(const __nv_bfloat16 *H, int64_t streams, int64
         prefix_stream_kernel<<<dim3((unsigned)streams, (unsigned)((D * D / 4 + 255) / 256)), 256, 0, stream>>>(
             L.segs, L.P, state, D, c);
     }
-    const int grid = (int)std::min<int64_t>(ns, (int64_t)sms);
-    cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, L.P, L.Bscr, nullptr, N, (float)c,
-                                                                         dR, st);
-    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(L.segs, nullptr, L.Bscr, H, N, (float)c, dR,
-                                                                          st);
+    if (!launch_tmem_chol(H, N, ns, L, (float)c, dR, st, stream)) return DBC_ERR_CUDA;
     count_launches(fused ? 4 : 5);
     return launch_status();
 }

@@ -28,6 +28,8 @@
 //    place, and the excess of each column gives dR_t = log1p(e_t) / 2.
 #pragma once
 
+#include <cuda.h>
+
 #include "tc.cuh"
 
 namespace dbc {
@@ -137,15 +139,19 @@ __device__ __forceinline__ void ypair(int pi, int &c, int &k) {
     while (k > c) { k -= c + 1; ++c; }
 }
 
+// tmP: P as fp32 [segments * 256][256] in 32 x 32 boxes (128-byte swizzle); tmB: B's pieces as bf16
+// [segments * 3 * 256][256] in 64 x 64 boxes (128-byte swizzle).  Both cover this GPU's own memory;
+// the factor mode loads P and stores B through them, the in-segment mode does not use them.
 template <bool FACTOR>
 __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
-    Segs S, const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr, const __nv_bfloat16 *__restrict__ Hx,
-    int64_t N, float c_rate, float *dR, int32_t *st) {
+    const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmB, Segs S,
+    const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr, const __nv_bfloat16 *__restrict__ Hx, int64_t N,
+    float c_rate, float *dR, int32_t *st) {
     constexpr int D = 256;
     extern __shared__ uint8_t smraw[];
     // [0], [1] panel MMA groups; [2] the final drain; [3], [4] Y operand stages consumed; [5] Y chunk done;
     // [6], [7] Y operand stages loaded (one arrival from each of the 224 loading threads)
-    __shared__ uint64_t mbar[8];
+    __shared__ uint64_t mbar[9];                    // [8]: the factor mode's P boxes landed
     __shared__ uint32_t tmem_base;
     __shared__ __align__(16) float s_LdT[16][16];   // factored 16 x 16 diagonal block, column-major
     __shared__ __align__(16) float s_rl[16];        // 1 / L_kk of the diagonal block
@@ -161,6 +167,11 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) tc::mbar_init(&mbar[i], 1);
+        tc::mbar_init(&mbar[8], 1);
+        if (FACTOR) {
+            tc::tma_prefetch_desc(&tmP);
+            tc::tma_prefetch_desc(&tmB);
+        }
         for (int i = 6; i < 8; ++i) tc::mbar_init(&mbar[i], 7 * 32);
         tc::fence_mbar_init();
     }
@@ -179,6 +190,7 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
         const uint32_t trow = tbase + ((uint32_t)lb << 16) + (uint32_t)(blk * 256);
         uint32_t ph0 = 0, ph1 = 0;      // mbarrier phases (uniform across the compute threads)
         uint32_t phs = 0, phy = 0, pf = 0;   // phs, pf: bit q = parity of the next wait on stage q
+        uint32_t pph = 0;                    // parity of the next wait on the P boxes
         bool ok = true;
         // A timeout makes `ok` false: every later wait and MMA is skipped (commits still arrive),
         // and the block-wide votes keep all threads on the same path to the end.
@@ -189,42 +201,41 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
 
             // ---------------- load the matrix into TMEM
             if (FACTOR) {
-                // each thread moves its own row of the c-scaled prefix Gram into TMEM: the lower
-                // triangle (loaded straight from global memory, 32-column chunks double-buffered in
-                // registers so that two chunks' loads are in flight) and zeros right of it, where
-                // B = L^{-T} accumulates
-                const float *P = Pbuf + (size_t)s * D * D + (size_t)row * D;
-                auto ldq = [&](int q, float4 (&x)[8]) {
-                    if (q * 32 <= row) {                                 // warp-uniform
+                // The c-scaled prefix Gram's lower triangle at 32-column granularity comes in with TMA:
+                // box (q, rb) = rows rb*32 .. +31 x columns q*32 .. +31 for rb >= q, 36 boxes of 4 KB,
+                // all in flight at once, in slots ordered by q then rb.  Each thread then moves its own
+                // row into TMEM (zeros right of its diagonal, where B = L^{-T} accumulates).
+                auto slot = [](int q, int rb) { return 8 * q - (q * (q - 1)) / 2 + (rb - q); };
+                if (tid == 0 && ok) {
+                    tc::mbar_arrive_expect_tx(&mbar[8], 36u * 4096u);
+                    for (int q = 0; q < 8; ++q)
+                        for (int rb = q; rb < 8; ++rb)
+                            tc::tma_load_2d(region + (uint32_t)slot(q, rb) * 4096u, &tmP, &mbar[8], q * 32,
+                                            s * D + rb * 32);
+                }
+                if (ok) ok = tc::mbar_wait(&mbar[8], pph, st);
+                pph ^= 1u;
+                const uint8_t *pbox = smraw + (region - tc::smem_u32(smraw));
+                const int rb = row >> 5, rin = row & 31;
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    const bool any = ok && q <= rb;                    // warp-uniform
+                    float x[32];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) x[i] = *reinterpret_cast<const float4 *>(P + q * 32 + 4 * i);
+                    for (int c = 0; c < 8; ++c) {
+                        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (any)
+                            f = *reinterpret_cast<const float4 *>(pbox + (size_t)slot(q, rb) * 4096 + rin * 128 +
+                                                                  ((c ^ (rin & 7)) * 16));
+                        x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
                     }
-                };
-                auto stq = [&](int q, const float4 (&x)[8]) {
-                    const bool any = q * 32 <= row;
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         float v[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int col = q * 32 + j * 16 + i;
-                            const float4 &f = x[(j * 16 + i) >> 2];
-                            const float e = ((i & 3) == 0) ? f.x : ((i & 3) == 1) ? f.y : ((i & 3) == 2) ? f.z : f.w;
-                            v[i] = (any && col <= row) ? e : 0.f;
-                        }
+                        for (int i = 0; i < 16; ++i) v[i] = (q * 32 + j * 16 + i <= row) ? x[j * 16 + i] : 0.f;
                         tc::tmem_st16(trow + (uint32_t)(q * 32 + j * 16), v);
                     }
-                };
-                float4 xa[8], xb[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) xa[i] = xb[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                ldq(0, xa);
-#pragma unroll 1
-                for (int q = 0; q < D / 32; q += 2) {
-                    ldq(q + 1, xb);
-                    stq(q, xa);
-                    if (q + 2 < D / 32) ldq(q + 2, xa);
-                    stq(q + 1, xb);
                 }
                 tc::tmem_wait_st();
             } else {
@@ -585,13 +596,13 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
             if (FACTOR && ok) {
                 // B = L^{-T} (TMEM upper triangle with the diagonal) -> three bf16 pieces in global
                 // memory, 64 columns at a time: each thread splits its row (zero left of the diagonal)
-                // into shared memory (row-major, 16-byte chunks XOR-swizzled by row), then warps copy
-                // whole 128-byte row pieces out.  Rows below a chunk's last panel are never read by the
-                // whitening loads and are not stored.
-                __nv_bfloat16 *Bs = Bscr + (size_t)s * 3 * D * D;
-                uint8_t *stg = smraw + (region - tc::smem_u32(smraw));
+                // into shared memory in the 128-byte swizzled layout of a 64 x 64 box (alternating
+                // between two staging buffers), and one thread stores the boxes with TMA.  Rows below
+                // a chunk's last panel are never read by the whitening loads and are not stored.
 #pragma unroll 1
                 for (int q = 0; q < D / 64; ++q) {
+                    const uint32_t stgb = region + (uint32_t)(q & 1) * (3u * 256u * 128u);
+                    uint8_t *stg = smraw + (stgb - tc::smem_u32(smraw));
 #pragma unroll 1
                     for (int h = 0; h < 4; ++h) {
                         float v16[16];
@@ -614,16 +625,25 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                                 make_uint4(ll[4 * c2], ll[4 * c2 + 1], ll[4 * c2 + 2], ll[4 * c2 + 3]);
                         }
                     }
+                    tc::fence_async_smem();
                     cbar();
-                    const int nrows = min(D, q * 64 + 64);                 // rows that hold B in this chunk
-                    for (int e = tid; e < 3 * nrows * 8; e += 256) {
-                        const int p = e / (nrows * 8), rest = e - p * nrows * 8, r = rest >> 3, c = rest & 7;
-                        const uint4 val = *reinterpret_cast<const uint4 *>(stg + (size_t)p * 256 * 128 + (size_t)r * 128 +
-                                                                           ((c ^ (r & 7)) * 16));
-                        *reinterpret_cast<uint4 *>(Bs + (size_t)p * D * D + (size_t)r * D + q * 64 + c * 8) = val;
+                    if (tid == 0) {
+                        for (int p = 0; p < 3; ++p)
+                            for (int rbk = 0; rbk <= q; ++rbk)
+                                asm volatile(
+                                    "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+                                    ::"l"(&tmB), "r"(q * 64), "r"((s * 3 + p) * D + rbk * 64),
+                                    "r"(stgb + (uint32_t)p * 256u * 128u + (uint32_t)rbk * 64u * 128u)
+                                    : "memory");
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        // the stores of the previous chunk have read their buffer, which the next chunk
+                        // refills
+                        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
                     }
                     cbar();
                 }
+                if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // region reused next
+                cbar();
             }
         }
     }
