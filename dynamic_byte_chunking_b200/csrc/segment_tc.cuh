@@ -517,16 +517,18 @@ inline bool launch_gram_prefix(const __nv_bfloat16 *H, int64_t N, int64_t rows, 
 inline bool launch_tmem_chol(const __nv_bfloat16 *H, int64_t N, int64_t ns, const Layout3 &L, float c, float *dR,
                              int32_t *st, cudaStream_t stream) {
     constexpr int D = 256;
-    CUtensorMap tmP, tmB;
+    CUtensorMap tmP, tmB, tmX;
     if (!tma::encode_f32_rows(&tmP, L.P, (uint64_t)ns * D, D, 32)) return false;
     if (!tma::encode_bf16_rows(&tmB, L.Bscr, (uint64_t)ns * 3 * D, D, 64)) return false;
+    const int xbox = (int)std::min<int64_t>(N, 256);
+    if (!tma::encode_bf16_rows(&tmX, H, (uint64_t)N, D, (uint32_t)xbox)) return false;
     const int grid = (int)std::min<int64_t>(ns, (int64_t)num_sms());
     cudaFuncSetAttribute(tmem_chol_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
     cudaFuncSetAttribute(tmem_chol_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TmemChol::SMEM);
-    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(tmP, tmB, L.segs, L.P, L.Bscr, nullptr, N, c,
-                                                                         dR, st);
-    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(tmP, tmB, L.segs, nullptr, L.Bscr, H, N, c,
-                                                                          dR, st);
+    tmem_chol_kernel<true><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(tmP, tmB, tmX, xbox, L.segs, L.P, L.Bscr, nullptr,
+                                                                         N, c, dR, st);
+    tmem_chol_kernel<false><<<grid, TmemChol::NT, TmemChol::SMEM, stream>>>(tmP, tmB, tmX, xbox, L.segs, nullptr, L.Bscr, H,
+                                                                          N, c, dR, st);
     return true;
 }
 

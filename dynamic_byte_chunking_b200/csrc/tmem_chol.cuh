@@ -140,17 +140,19 @@ __device__ __forceinline__ void ypair(int pi, int &c, int &k) {
 }
 
 // tmP: P as fp32 [segments * 256][256] in 32 x 32 boxes (128-byte swizzle); tmB: B's pieces as bf16
-// [segments * 3 * 256][256] in 64 x 64 boxes (128-byte swizzle).  Both cover this GPU's own memory;
-// the factor mode loads P and stores B through them, the in-segment mode does not use them.
+// [segments * 3 * 256][256] in 64 x 64 boxes (128-byte swizzle); tmX: H as bf16 [N][256] in boxes of
+// xbox_rows = min(N, 256) positions x 64 features (128-byte swizzle).  All cover this GPU's own memory (no multicast):
+// the factor mode loads P and stores B through them, the in-segment mode loads X and B.
 template <bool FACTOR>
 __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
-    const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmB, Segs S,
+    const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmB,
+    const __grid_constant__ CUtensorMap tmX, int xbox_rows, Segs S,
     const float *__restrict__ Pbuf, __nv_bfloat16 *Bscr, const __nv_bfloat16 *__restrict__ Hx, int64_t N,
     float c_rate, float *dR, int32_t *st) {
     constexpr int D = 256;
     extern __shared__ uint8_t smraw[];
     // [0], [1] panel MMA groups; [2] the final drain; [3], [4] Y operand stages consumed; [5] Y chunk done;
-    // [6], [7] Y operand stages loaded (one arrival from each of the 224 loading threads)
+    // [6], [7] Y operand stages loaded (TMA bytes)
     __shared__ uint64_t mbar[9];                    // [8]: the factor mode's P boxes landed
     __shared__ uint32_t tmem_base;
     __shared__ __align__(16) float s_LdT[16][16];   // factored 16 x 16 diagonal block, column-major
@@ -168,11 +170,9 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) tc::mbar_init(&mbar[i], 1);
         tc::mbar_init(&mbar[8], 1);
-        if (FACTOR) {
-            tc::tma_prefetch_desc(&tmP);
-            tc::tma_prefetch_desc(&tmB);
-        }
-        for (int i = 6; i < 8; ++i) tc::mbar_init(&mbar[i], 7 * 32);
+        tc::tma_prefetch_desc(FACTOR ? &tmP : &tmX);
+        tc::tma_prefetch_desc(&tmB);
+        for (int i = 6; i < 8; ++i) tc::mbar_init(&mbar[i], 1);
         tc::fence_mbar_init();
     }
     tc::fence_before_sync();
@@ -245,50 +245,33 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 // k <= c (B is upper triangular) with X and the three pieces of B streamed through
                 // two cp.async stages; Y_c is then split into three bf16 pieces in shared memory and
                 // G' += Y_c Y_c^T (six piece products) is issued while the next chunk's operands load.
-                const __nv_bfloat16 *Xs = Hx + start * D;
-                const __nv_bfloat16 *Bseg = Bscr + (size_t)s * 3 * D * D;
-                auto load = [&](int pi, uint32_t sa) {
+                // The issuing thread loads the operand stages with TMA: X_s's 256 positions x 64
+                // features of K chunk k (one box; positions past the segment, whose Y rows never reach
+                // the leading n x n block that is factored, arrive too, or as zeros past the end of H)
+                // and the three pieces of B's 64 x 64 block (k, c), every one of which the factor mode
+                // stored.
+                auto tload = [&](int pi, int q) {
                     int c, k;
                     ypair(pi, c, k);
-                    for (int e = tid; e < 256 * 8; e += 7 * 32) {           // X: 256 positions x 64 K
-                        const int r = e >> 3, ch = e & 7;
-                        const bool in = r < len;
-                        const uint32_t xo =
-                            (r < 128) ? tc::kmajor_off(r, ch * 8) : 128 * 128 + tc::kmajor_off(r - 128, ch * 8);
-                        tc::cp_async16(sa + xo, Xs + (size_t)(in ? r : 0) * D + k * 64 + ch * 8, in ? 16u : 0u);
-                    }
-                    const uint32_t sb = sa + TmemChol::YX_BYTES;
-                    for (int e = tid; e < 3 * 64 * 8; e += 7 * 32) {        // B: 3 pieces x 64 K x 64 N
-                        const int p = e >> 9, kr = (e >> 3) & 63, n8 = e & 7;
-                        const int krow = k * 64 + kr, col = c * 64 + n8 * 8;
-                        const bool nz = krow < (col >> 4) * 16 + 16;         // stored rows of the columns' panel
-                        tc::cp_async16(sb + (uint32_t)p * 8192 + tc::mnmajor_off(n8 * 8, kr, 8192),
-                                       Bseg + (size_t)p * D * D + (size_t)(nz ? krow : 0) * D + col, nz ? 16u : 0u);
-                    }
+                    const uint32_t sa = region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE;
+                    tc::mbar_arrive_expect_tx(&mbar[6 + q], (uint32_t)xbox_rows * 128u + 3u * 8192u);
+                    tc::tma_load_2d(sa, &tmX, &mbar[6 + q], k * 64, (int)start);
+                    for (int p = 0; p < 3; ++p)
+                        tc::tma_load_2d(sa + TmemChol::YX_BYTES + (uint32_t)p * 8192u, &tmB, &mbar[6 + q], c * 64,
+                                        (s * 3 + p) * D + k * 64);
                 };
                 const float sc = sqrtf(c_rate);
-                // warps 0..6 stream the operand stages and announce each on full[stage]; warp 7 only
-                // issues (its lane 0) and joins the Y_c read-outs, so a long MMA issue (G' takes a
-                // few thousand cycles) never holds up the next stage's loads
-                const bool loader = warp < 7;
-                if (loader) load(0, region + TmemChol::YSTAGE0);
-                tc::cp_async_commit();
+                if (issuer && ok) tload(0, 0);
                 for (int pi = 0; pi < NPAIR; ++pi) {
                     int c, k;
                     ypair(pi, c, k);
                     if (pi + 1 < NPAIR) {
                         const int q = (pi + 1) & 1;
                         if (pi + 1 >= 2) {                                   // stage q was read by pair pi - 1
-                            if (loader && ok) ok = tc::mbar_wait(&mbar[3 + q], (phs >> q) & 1u, st);
+                            if (issuer && ok) ok = tc::mbar_wait(&mbar[3 + q], (phs >> q) & 1u, st);
                             phs ^= 1u << q;
                         }
-                        if (loader) load(pi + 1, region + TmemChol::YSTAGE0 + (uint32_t)q * TmemChol::YSTAGE);
-                    }
-                    tc::cp_async_commit();
-                    if (loader) {
-                        tc::cp_async_wait<1>();
-                        tc::fence_async_smem();
-                        tc::mbar_arrive(&mbar[6 + (pi & 1)]);            // stage pi is in place
+                        if (issuer && ok) tload(pi + 1, q);
                     }
                     if (issuer) {
                         if (ok) ok = tc::mbar_wait(&mbar[6 + (pi & 1)], (pf >> (pi & 1)) & 1u, st);
