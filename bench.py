@@ -246,26 +246,30 @@ def write_traffic(csv_path):
 
 
 def stage_rooflines(avg_ms, N, d, rows, K, nb, pk, src):
-    """Achieved / peak of every stage of the step from its event-timed average duration.
+    """Achieved / peak of every stage of the step from its event-timed average duration (avg_ms: stage
+    name -> ms per call).
 
     Algorithmic work per call: coding rate 4 d^2 N flop (the rank-1 recursion: 2 d^2 for the solve and
     2 d^2 for the update per position) against the bf16 tensor peak; Top-K, gather and upsample their
-    compulsory HBM bytes (read inputs once, write outputs once) against the HBM copy bandwidth."""
+    compulsory HBM bytes (read inputs once, write outputs once) against the HBM
+    copy bandwidth."""
     flops_cr = 4.0 * d * d * N
     tf = pk.get("bf16_tflops", 1590.0)
     hbm = pk.get("hbm_gbs", 6650.0)
     out = {}
-    a = flops_cr / (avg_ms[0] * 1e-3) / 1e12
-    out["chunk_coding_rate"] = {"bound": "tensor", "achieved": a, "peak": tf, "unit": "TFLOP/s", "frac": a / tf,
-                                "algorithmic": f"4*d^2*N = {flops_cr:.4g} flop per call",
-                                "peak_source": src + " bf16 (burst)"}
     by = {"chunk_topk_select": N * 4 + rows * K * 8 + (rows + 1) * 8,          # read dR, write idx
           "chunk_gather": 2 * rows * K * d * 2,                                 # read + write chunk rows
           "chunk_upsample": N * d * 2 + rows * K * d * 2 + nb * d * d * 2 + N * d * 4}   # H, G, W in; S out
-    for i, st in enumerate(["chunk_topk_select", "chunk_gather", "chunk_upsample"], start=1):
-        g = by[st] / (avg_ms[i] * 1e-3) / 1e9
-        out[st] = {"bound": "hbm", "achieved": g, "peak": hbm, "unit": "GB/s", "frac": g / hbm,
-                   "algorithmic": f"{by[st]} bytes per call", "peak_source": src}
+    for st, ms in avg_ms.items():
+        if st == "chunk_coding_rate":
+            a = flops_cr / (ms * 1e-3) / 1e12
+            out[st] = {"bound": "tensor", "achieved": a, "peak": tf, "unit": "TFLOP/s", "frac": a / tf,
+                       "algorithmic": f"4*d^2*N = {flops_cr:.4g} flop per call",
+                       "peak_source": src + " bf16 (burst)"}
+        else:
+            g = by[st] / (ms * 1e-3) / 1e9
+            out[st] = {"bound": "hbm", "achieved": g, "peak": hbm, "unit": "GB/s", "frac": g / hbm,
+                       "algorithmic": f"{by[st]} bytes per call", "peak_source": src}
     return out
 
 
@@ -566,23 +570,25 @@ def main():
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
 
+    # the step: the four calls
+    calls = {
+        "chunk_coding_rate": lambda Hx: dbc.chunk_coding_rate(Hx, w.eps2, dR=dR, workspace=ws_cr, dev_status=st),
+        "chunk_topk_select": lambda Hx: dbc.chunk_topk_select(dR, K, rows=rows, T=T, idx=idx, idx_offsets=io,
+                                                              dev_status=st),
+        "chunk_gather": lambda Hx: dbc.chunk_gather(Hx, idx, io, rows=rows, T=T, total=rows * K, Z=Z,
+                                                    dev_status=st),
+        "chunk_upsample": lambda Hx: dbc.chunk_upsample(Z, Hx, idx, io, Wb, rows=rows, T=T, S=S, workspace=ws_up,
+                                                        dev_status=st)}
     stages = ["chunk_coding_rate", "chunk_topk_select", "chunk_gather", "chunk_upsample"]
+    ns_ = len(stages)
 
     def step(Hx, ev=None):
+        for i, name in enumerate(stages):
+            if ev is not None:
+                ev[i].record(stream)
+            calls[name](Hx)
         if ev is not None:
-            ev[0].record(stream)
-        dbc.chunk_coding_rate(Hx, w.eps2, dR=dR, workspace=ws_cr, dev_status=st)
-        if ev is not None:
-            ev[1].record(stream)
-        dbc.chunk_topk_select(dR, K, rows=rows, T=T, idx=idx, idx_offsets=io, dev_status=st)
-        if ev is not None:
-            ev[2].record(stream)
-        dbc.chunk_gather(Hx, idx, io, rows=rows, T=T, total=rows * K, Z=Z, dev_status=st)
-        if ev is not None:
-            ev[3].record(stream)
-        dbc.chunk_upsample(Z, Hx, idx, io, Wb, rows=rows, T=T, S=S, workspace=ws_up, dev_status=st)
-        if ev is not None:
-            ev[4].record(stream)
+            ev[ns_].record(stream)
 
     def check_status(when):
         # collective, so that every rank stops together when any rank saw a device flag
@@ -604,17 +610,12 @@ def main():
     graphs, per_step_launches, launch_mode = None, None, "eager"
     if not args.no_graph:
         try:
-            calls = [
-                lambda: dbc.chunk_coding_rate(H, w.eps2, dR=dR, workspace=ws_cr, dev_status=st),
-                lambda: dbc.chunk_topk_select(dR, K, rows=rows, T=T, idx=idx, idx_offsets=io, dev_status=st),
-                lambda: dbc.chunk_gather(H, idx, io, rows=rows, T=T, total=rows * K, Z=Z, dev_status=st),
-                lambda: dbc.chunk_upsample(Z, H, idx, io, Wb, rows=rows, T=T, S=S, workspace=ws_up, dev_status=st)]
             l0 = dbc.launch_count()
             graphs = []
-            for c in calls:
+            for name in stages:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
-                    c()
+                    calls[name](H)
                 graphs.append(g)
             per_step_launches = dbc.launch_count() - l0
             torch.cuda.synchronize()
@@ -637,9 +638,9 @@ def main():
         for s_, g in enumerate(graphs):
             ev[s_].record(stream)
             g.replay()
-        ev[4].record(stream)
+        ev[ns_].record(stream)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ns_ + 1)] for _ in range(args.steps)]
     gpu_id = str(local)
     try:
         props = torch.cuda.get_device_properties(dev)
@@ -664,12 +665,12 @@ def main():
     time.sleep(0.2)
     clocks = sampler.stop()
 
-    per_stage = np.zeros(4)
+    per_stage = np.zeros(ns_)
     total = 0.0
     for e in evs:
-        for s in range(4):
+        for s in range(ns_):
             per_stage[s] += e[s].elapsed_time(e[s + 1])
-        total += e[0].elapsed_time(e[4])
+        total += e[0].elapsed_time(e[ns_])
     t_ms = torch.tensor([total], dtype=torch.float64, device=dev)
     if pg:
         pg.all_reduce(t_ms, op=pg.ReduceOp.MAX)
@@ -680,13 +681,13 @@ def main():
     # ---- roofline of every stage, and of the dominant one (the coding-rate call)
     pk, src = peaks()
     avg = per_stage / args.steps          # ms per call
-    stage_roof = stage_rooflines(avg, N, d, rows, K, nb, pk, src)
+    stage_roof = stage_rooflines(dict(zip(stages, avg)), N, d, rows, K, nb, pk, src)
     dom = int(np.argmax(avg))
     roof = dict(stage_roof[stages[dom]])
     roof["traffic"] = stored_traffic(stages[dom])
     roof["kernel"] = stages[dom]
     # the metric's own definition: positions / (coding rate + Top-K + gather)
-    t_chunk = float(avg[0] + avg[1] + avg[2])
+    t_chunk = float(sum(a_ for s_, a_ in zip(stages, avg) if s_ != "chunk_upsample"))
     value_chunk = N * world / (t_chunk * 1e-3)
 
     # ---- end to end through host buffers: every step copies its H from pinned host memory to the
@@ -775,7 +776,7 @@ def main():
                            "step": " -> ".join(stages), "launch": launch_mode},
                 "stage_ms": {s: float(a) for s, a in zip(stages, avg)},
                 "value_chunk": {"value": value_chunk, "unit": UNIT, "ms": t_chunk,
-                                "definition": "positions / (chunk_coding_rate + chunk_topk_select + chunk_gather)"},
+                                "definition": "positions / (coding rate + Top-K + gather)"},
                 "stage_roofline": stage_roof,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
                 "clocks": clocks}

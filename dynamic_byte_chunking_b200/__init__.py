@@ -26,7 +26,7 @@ from typing import Optional
 __all__ = [
     "DbcError", "lib", "lib_path", "version", "status_string", "launch_count",
     "chunk_coding_rate", "chunk_coding_rate_workspace", "chunk_coding_rate_stream",
-    "chunk_coding_rate_stream_workspace", "chunk_topk_select", "chunk_topk_select_gather",
+    "chunk_coding_rate_stream_workspace", "chunk_topk_select",
     "chunk_gather", "chunk_upsample", "chunk_upsample_workspace", "chunk_upsample_noalloc",
     "chunk_upsample_backward", "chunk_upsample_backward_workspace", "chunk_gather_backward",
     "hnet_route", "hnet_route_workspace", "chunk", "canon_conv1d", "chunk_coding_rate_canon",
@@ -55,8 +55,6 @@ _SIGS = {
     "chunk_coding_rate_stream": (_int, [_vp, _int, _i64, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "chunk_topk_select_workspace": (_sz, [_i64]),
     "chunk_topk_select": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
-    "chunk_topk_select_gather": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _i64, _i64,
-                                        _vp, _vp, _vp]),
     "chunk_gather": (_int, [_vp, _int, _vp, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp,
                             _vp, _vp]),
     "chunk_upsample_workspace": (_sz, [_i64, _i64, _int]),
@@ -247,37 +245,6 @@ def chunk_topk_select(dR, K, *, rows: int, T: int, offsets=None, total: Optional
     if total is not None:
         idx = idx[:total]
     return idx, idx_offsets
-
-
-def chunk_topk_select_gather(dR, K, H, *, rows: int, T: int, offsets=None, total: Optional[int] = None,
-                             idx=None, idx_offsets=None, Z=None, dev_status=None, stream=None):
-    """(idx, idx_offsets, Z): chunk_topk_select and chunk_gather (no projection) in one launch."""
-    torch = _torch()
-    _require_cuda(dR, H, offsets)
-    N = dR.numel()
-    H2 = H.reshape(-1, H.shape[-1]).contiguous()
-    d = H2.shape[1]
-    Kp, Ks = (K, 0) if torch.is_tensor(K) else (None, int(K))
-    if Kp is not None:
-        _require_cuda(Kp)
-    if total is None:
-        if idx is not None:
-            total = idx.numel()
-        elif Kp is not None or offsets is not None:
-            raise ValueError("pass `total` (or a preallocated idx) with ragged rows or per-row K")
-        else:
-            total = rows * min(Ks, T)
-    if idx is None:
-        idx = torch.empty(max(total, 1), dtype=torch.int64, device=dR.device)
-    if idx_offsets is None:
-        idx_offsets = torch.empty(rows + 1, dtype=torch.int64, device=dR.device)
-    if Z is None:
-        Z = torch.empty(max(total, 1), d, dtype=H.dtype, device=H.device)
-    rc = lib().chunk_topk_select_gather(_ptr(dR), _ptr(offsets), rows, T, N, _ptr(Kp), Ks, _ptr(idx),
-                                        _ptr(idx_offsets), _ptr(H2), _dtype_code(H2), d, total, _ptr(Z),
-                                        _ptr(dev_status), _stream(stream))
-    _check("chunk_topk_select_gather", rc)
-    return idx[:total], idx_offsets, Z[:total]
 
 
 def chunk_gather(H, idx, idx_offsets, *, rows: int, T: int, offsets=None, total: Optional[int] = None,

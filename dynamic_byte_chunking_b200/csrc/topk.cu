@@ -277,28 +277,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float *__restric
 
 
 // ---------------------------------------------------------------- cluster per row
-// The chunk vectors of output slots [o0, o1) of one row (H rows a + out[o] -> Z rows obase + o), one
-// warp per four rows per step with every 16-byte load of the four rows in flight before the stores.
-// out[] was written by this CTA before the barrier that precedes the call.
-__device__ __forceinline__ void copy_rows(const int64_t *out, int64_t o0, int64_t o1, int64_t a, int64_t obase,
-                                          const uint4 *__restrict__ H, int64_t vec, uint4 *__restrict__ Z,
-                                          int nthreads) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = nthreads >> 5;
-    for (int64_t o = o0 + 4 * w; o < o1; o += 4 * nw) {
-        int64_t src[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) src[q] = o + q < o1 ? (a + out[o + q]) * vec : -1;
-        for (int64_t v = lane; v < vec; v += 32) {
-            uint4 val[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) val[q] = src[q] >= 0 ? H[src[q] + v] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (src[q] >= 0) Z[(obase + o + q) * vec + v] = val[q];
-        }
-    }
-}
-
 constexpr int kCluster = 8;
 constexpr int kCThreads = 256;
 constexpr int kCWarps = kCThreads / 32;
@@ -308,7 +286,7 @@ constexpr int kClusterKeys = kCluster * kSliceKeys;    // candidates per row on 
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     select_cluster_kernel(const float *__restrict__ dR, const int64_t *offsets, int64_t rows, int64_t T,
                           const int64_t *Kp, int64_t Ks, int64_t dense_K, int64_t *idx_offsets, int64_t *idx,
-                          const uint4 *__restrict__ H, int64_t vec_per_row, uint4 *__restrict__ Z, int32_t *st) {
+                          int32_t *st) {
     __shared__ uint32_t keys[kSliceKeys];
     __shared__ uint32_t hist[2][256];                  // alternate passes: a pass never clears what is read
     __shared__ uint32_t tot[256];
@@ -339,19 +317,9 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     if (n <= 0) return;
     if (K >= n) {
         for (int64_t t = (int64_t)q * kCThreads + tid; t < n; t += kCluster * kCThreads) out[t] = t;
-        if (Z) {
-            // every position: slot t holds position t (this CTA's share of the rows)
-            const int64_t per = (n + kCluster - 1) / kCluster;
-            const int64_t t0 = (int64_t)q * per, t1 = min(n, t0 + per);
-            const int lane = tid & 31, w = tid >> 5;
-            for (int64_t t = t0 + w; t < t1; t += kCWarps)
-                for (int64_t v = lane; v < vec_per_row; v += 32) Z[(obase + t) * vec_per_row + v] = H[(a + t) * vec_per_row + v];
-        }
         return;
     }
     if (q == 0 && tid == 0) out[0] = 0;
-    if (Z && q == 0 && tid < 32)
-        for (int64_t v = tid; v < vec_per_row; v += 32) Z[obase * vec_per_row + v] = H[a * vec_per_row + v];
     const int need = (int)(K - 1);
     if (need == 0) return;
     const int m = (int)(n - 1);                        // candidates t = 1 .. n-1 (m <= kClusterKeys)
@@ -459,12 +427,6 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     }
     // this CTA's reads of the other slices' counts are done; its own may still be read
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    // this slice's outputs: slots 1 + slice_before .. + slice_count
-    const int slice_before = sel_before;
-    const int slice_count = s_cnt[1] + [&] {
-        const int l = rem - eq_before, e = s_cnt[0];
-        return l <= 0 ? 0 : (l >= e ? e : l);
-    }();
     for (int w = 0; w < wid; ++w) {
         const int e = s_weq[w], g = s_wgt[w];
         const int l = rem - eq_before;
@@ -488,12 +450,6 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
         }
         o += __popc(sm);
         eq_run += __popc(em);
-    }
-    if (Z) {
-        // the chunk vectors of this slice's outputs, whose positions every warp of this CTA wrote above
-        __syncthreads();
-        copy_rows(out, 1 + (int64_t)slice_before, 1 + (int64_t)slice_before + slice_count, a, obase, H, vec_per_row,
-                  Z, kCThreads);
     }
     // no CTA leaves while its counts may still be read
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -533,7 +489,7 @@ extern "C" dbc_status chunk_topk_select(const float *dR, const int64_t *offsets,
     if (m <= tk::kClusterKeys && rows <= INT32_MAX / tk::kCluster) {
         // every row fits the cluster path (T is the longest row)
         tk::select_cluster_kernel<<<(unsigned)(rows * tk::kCluster), tk::kCThreads, 0, s>>>(
-            dR, offsets, rows, T, K_per_row, K_scalar, dense_K, idx_offsets, idx, nullptr, 0, nullptr, dev_status);
+            dR, offsets, rows, T, K_per_row, K_scalar, dense_K, idx_offsets, idx, dev_status);
         count_launches(1);
         return launch_status();
     }
@@ -543,41 +499,6 @@ extern "C" dbc_status chunk_topk_select(const float *dR, const int64_t *offsets,
     const int grid = (int)std::min<int64_t>(rows, 65535);
     tk::select_kernel<<<grid, tk::kThreads, smem, s>>>(dR, offsets, rows, T, K_per_row, K_scalar, dense_K,
                                                        idx_offsets, idx, keys, dev_status);
-    count_launches(1);
-    return launch_status();
-}
-
-extern "C" dbc_status chunk_topk_select_gather(const float *dR, const int64_t *offsets, int64_t rows, int64_t T,
-                                               int64_t N, const int64_t *K_per_row, int64_t K_scalar, int64_t *idx,
-                                               int64_t *idx_offsets, const void *H, int dtype, int64_t d,
-                                               int64_t total_K, void *Z, int32_t *dev_status, dbc_stream_t stream) {
-    DBC_NVTX_RANGE("chunk_topk_select_gather");
-    if (rows < 0 || T < 0 || N < 0 || d <= 0 || total_K < 0) return DBC_ERR_INVALID_ARG;
-    if (!K_per_row && K_scalar < 1) return DBC_ERR_INVALID_ARG;
-    if (!offsets && N != rows * T) return DBC_ERR_INVALID_ARG;
-    if (!idx_offsets) return DBC_ERR_INVALID_ARG;
-    if (dtype != DBC_F32 && dtype != DBC_BF16) return DBC_ERR_UNSUPPORTED;
-    const int64_t esz = dtype == DBC_BF16 ? 2 : 4;
-    if ((d * esz) % 16) return DBC_ERR_UNSUPPORTED;
-    if (rows > 0 && N > 0 && (!dR || !idx || !H || !Z || !aligned16(H) || !aligned16(Z))) return DBC_ERR_INVALID_ARG;
-    const int64_t m = T > 1 ? T - 1 : 1;
-    if (rows == 0 || N == 0 || m > tk::kClusterKeys || rows > INT32_MAX / tk::kCluster) {
-        // the two calls one after the other (long rows, or nothing to do)
-        const dbc_status e = chunk_topk_select(dR, offsets, rows, T, N, K_per_row, K_scalar, idx, idx_offsets,
-                                               nullptr, 0, dev_status, stream);
-        if (e != DBC_OK || rows == 0 || N == 0) return e;
-        return chunk_gather(H, dtype, offsets, T, d, idx, idx_offsets, rows, total_K, Z, nullptr, 0, nullptr, nullptr,
-                            dev_status, stream);
-    }
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t dense_K = (!offsets && !K_per_row) ? K_scalar : 0;
-    if (!dense_K) {
-        tk::offsets_kernel<<<1, 1024, 0, s>>>(offsets, rows, T, K_per_row, K_scalar, idx_offsets, dev_status);
-        count_launches(1);
-    }
-    tk::select_cluster_kernel<<<(unsigned)(rows * tk::kCluster), tk::kCThreads, 0, s>>>(
-        dR, offsets, rows, T, K_per_row, K_scalar, dense_K, idx_offsets, idx, static_cast<const uint4 *>(H),
-        d * esz / 16, static_cast<uint4 *>(Z), dev_status);
     count_launches(1);
     return launch_status();
 }

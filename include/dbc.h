@@ -178,26 +178,6 @@ DBC_API dbc_status chunk_gather(const void *H, int dtype, const int64_t *offsets
                         int32_t *dev_status, dbc_stream_t stream);
 
 /* -------------------------------------------------------------------------
- * chunk_topk_select_gather -- chunk_topk_select followed by chunk_gather (no
- * projection) in one launch: the boundary kernel copies each selected row
- * h_{s_k} into Z after writing s_k (ByteFlow notes "Key design 2"; summary
- * stage 2: boundaries, then z_k = h_{s_k}).
- *
- * Arguments as chunk_topk_select (dR, offsets, rows, T, N, K_per_row,
- * K_scalar, idx, idx_offsets) and chunk_gather (H of dtype, d, Z: [total_K,
- * d], H and Z 16-byte aligned, d * element size a multiple of 16 bytes);
- * total_K is the capacity of idx and Z in rows (>= sum_r min(K_r, T_r)).
- * The results are bit-identical to the two calls; rows longer than 65 537
- * positions run the two calls.  No workspace.
- * Errors: INVALID_ARG, UNSUPPORTED, CUDA; device flags as the two calls.
- * ------------------------------------------------------------------------- */
-DBC_API dbc_status chunk_topk_select_gather(const float *dR, const int64_t *offsets, int64_t rows,
-                                    int64_t T, int64_t N, const int64_t *K_per_row,
-                                    int64_t K_scalar, int64_t *idx, int64_t *idx_offsets,
-                                    const void *H, int dtype, int64_t d, int64_t total_K, void *Z,
-                                    int32_t *dev_status, dbc_stream_t stream);
-
-/* -------------------------------------------------------------------------
  * chunk_upsample -- multi-linear upsampling with residual.
  *
  * ByteFlow (summary stage 4; notes "Key design 4"): for each position t of a
