@@ -24,8 +24,10 @@
 //    M_s^{-1} = B B^T, the whitened rows Y = sqrt(c) X_s B give the segment's
 //    problem c X_s M_s^{-1} X_s^T = Y Y^T.
 //  * INSEG (one segment): G' = Y Y^T (Y in three pieces, six piece
-//    products) is accumulated straight into TMEM, I + G' is factored in
-//    place, and the excess of each column gives dR_t = log1p(e_t) / 2.
+//    products, or three products of the first two pieces for a 64-feature
+//    chunk of Y whose rows are all small) is accumulated straight into TMEM,
+//    I + G' is factored in place, and the excess of each column gives
+//    dR_t = log1p(e_t) / 2.
 #pragma once
 
 #include <cuda.h>
@@ -55,6 +57,14 @@ struct TmemChol {
     static constexpr uint32_t YREGION = YSTAGE0 + 2 * YSTAGE;
     static constexpr uint32_t REGION = (YREGION > 2 * PANEL) ? YREGION : 2 * PANEL;
     static constexpr size_t SMEM = REGION + 1024;
+    // A 64-feature chunk Y_c of G' = sum_c Y_c Y_c^T takes three of the six piece products
+    // (hi.hi, hi.mid, mid.hi: the two-piece split hi + mid, dropped terms below 2^-16 |y_t||y_u|)
+    // when every live row has |y_{t,c}|^2 <= this bound: each dropped entry is then below
+    // 2^-16 * 4 = 6e-5, far under the unit floor of I + G', so the leading factor's pivots move by
+    // a few parts in 1e5 (measured in float64 emulation on every workload family: dR within 2e-5
+    // relative).  Chunks above it (whitened rows the prefix has not yet explained: the first
+    // segments of a row) keep all six products.
+    static constexpr float Y2_TWO_PIECE = 4.f;
 };
 
 // Six piece products of a three-way split (dropped terms are below 2^-24):
@@ -126,6 +136,15 @@ __device__ __forceinline__ bool cbar_and(bool v) {
     uint32_t r;
     asm volatile(
         "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.and.pred p, 1, 256, q;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool cbar_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, 1, 256, q;\n selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(r)
         : "r"((uint32_t)v)
         : "memory");
@@ -301,25 +320,33 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                         phy ^= 1;
                         tc::fence_after_sync();
                         ok = __all_sync(0xffffffffu, ok);
+                        bool big = false;                  // this row's |Y_c|^2 above the two-piece bound
                         if (ok) {
                             float a64[64];
+                            float s2 = 0.f;
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
                                 float v16[16];
                                 tc::tmem_ld16(tbase + ((uint32_t)lb << 16) + (uint32_t)(128 + blk * 64 + q * 16), v16);
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) a64[q * 16 + i] = sc * v16[i];
+                                for (int i = 0; i < 16; ++i) {
+                                    a64[q * 16 + i] = sc * v16[i];
+                                    s2 = fmaf(a64[q * 16 + i], a64[q * 16 + i], s2);
+                                }
                             }
+                            big = row < n && !(s2 <= TmemChol::Y2_TWO_PIECE);
                             stage_row(region, row, a64, nullptr, 0);
                         }
                         tc::fence_async_smem();
                         tc::fence_before_sync();
                         ok = cbar_and(ok);
+                        const int npr = cbar_or(big) ? 6 : 3;
                         if (issuer && ok) {
                             tc::fence_after_sync();
                             const uint64_t dyp = tc::sdesc(region, 16, 1024);
 #pragma unroll
                             for (int pr = 0; pr < 6; ++pr) {
+                                if (pr >= npr) break;
                                 const uint32_t pa = (uint32_t)pair_a(pr) * TmemChol::PIECE;
                                 const uint32_t pb = (uint32_t)pair_b(pr) * TmemChol::PIECE;
 #pragma unroll

@@ -117,23 +117,45 @@ __global__ void __launch_bounds__(256) scatter_kernel(int64_t N, int nbins, Layo
 // K-major, cp.async by all threads), B = W_b (row-major [d_g][d_l], read
 // MN-major, TMA tile loads issued by one thread: tensor map over this GPU's own
 // memory, no multicast), fp32 accumulators in TMEM; the epilogue adds h_t and
-// scatters the rows back to their positions.
+// scatters the rows back to their positions.  Two stages of 48 KB keep the CTA
+// small enough for two per SM (with bf16 h), so one CTA's epilogue stores run
+// under the other's loads and MMAs.  The tile's residual values are loaded into
+// registers as soon as its positions are known, before anything else: each CTA
+// lives for one tile, so the DRAM reads it keeps in flight are what bounds the
+// kernel (issuing the second column half's loads only during the first half's
+// stores cost a quarter of the time on the ragged batch).
 struct BinTC {
-    static constexpr int NS = 3;
-    static constexpr uint32_t A_BYTES = 128 * 128;
+    static constexpr int NS = 2;
+    static constexpr uint32_t A_BYTES = 128 * 128;             // 128 rows x 64 K, K-major
     static constexpr uint32_t B_BYTES = 4 * 64 * 128;          // up to 256 columns x 64 K, MN-major
     static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
-    static constexpr uint32_t HBUF = 128 * 256 * 2;             // the tile's residual rows (bf16 H)
-    // bf16 H is prefetched into shared memory while the MMAs run; fp32 H is read in the epilogue
-    template <class IN>
-    static constexpr size_t smem() { return NS * STAGE + (sizeof(IN) == 2 ? HBUF : 0) + 1024; }
+    static constexpr int LDT = 132;                            // epilogue tile: [128][LDT] fp32, one column half
+    static_assert(128u * LDT * 4u <= NS * STAGE, "the epilogue tile reuses the stages");
+    static constexpr size_t SMEM = NS * STAGE + 1024;
+};
+
+// Four consecutive residual values of a row (8 bytes of bf16 or 16 of fp32).
+template <class IN> struct Res4;
+template <> struct Res4<__nv_bfloat16> {
+    using V = uint2;
+    static __device__ __forceinline__ V load(const __nv_bfloat16 *p) { return __ldg(reinterpret_cast<const uint2 *>(p)); }
+    static __device__ __forceinline__ void unpack(const V &v, float (&h)[4]) {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&v.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&v.y);
+        h[0] = __low2float(a); h[1] = __high2float(a); h[2] = __low2float(b); h[3] = __high2float(b);
+    }
+};
+template <> struct Res4<float> {
+    using V = float4;
+    static __device__ __forceinline__ V load(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+    static __device__ __forceinline__ void unpack(const V &v, float (&h)[4]) { h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w; }
 };
 
 template <class IN>
-__global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
-                                                             const __nv_bfloat16 *__restrict__ G, int64_t dg,
-                                                             const IN *__restrict__ H, int64_t dl, int nbins,
-                                                             Layout L, float *__restrict__ S, int64_t N, int32_t *st) {
+__global__ void __launch_bounds__(256, sizeof(IN) == 2 ? 2 : 1)
+    bin_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16 *__restrict__ G, int64_t dg,
+                       const IN *__restrict__ H, int64_t dl, int nbins, Layout L, float *__restrict__ S, int64_t N,
+                       int32_t *st) {
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar[BinTC::NS], wbar[BinTC::NS];      // stage consumed by the MMAs / W_b bytes landed
     __shared__ uint32_t tmem_base;
@@ -150,11 +172,7 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_consta
     const int64_t n0 = (int64_t)blockIdx.y * 256;
     const int nt = (int)(dl - n0 < 256 ? dl - n0 : 256);      // multiple of 64
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid < 128) {
-        const int p = tid < cnt ? L.perm[r0 + tid] : -1;
-        pos[tid] = p;
-        grow[tid] = p >= 0 ? L.chunk[p] : -1;
-    }
+    if (tid < 128) pos[tid] = tid < cnt ? L.perm[r0 + tid] : -1;
     const uint32_t base = (tc::smem_u32(smraw) + 1023u) & ~1023u;
     if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
     if (tid == 0) {
@@ -169,6 +187,27 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_consta
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = tmem_base;
+    // Residual of row (warp + 8 i), columns half * 128 + lane * 4 .. +3 (zeros for empty rows and
+    // columns past the tile): all of the tile's residual loads are issued here, before the chunk
+    // rows are looked up, and stay in flight through the MMAs
+    using R4 = Res4<IN>;
+    auto hload = [&](int half, int i) {
+        typename R4::V v{};
+        const int p = pos[warp + 8 * i];
+        const int col = half * 128 + lane * 4;
+        if (p >= 0 && p < N && col < nt) v = R4::load(H + (size_t)p * dl + n0 + col);
+        return v;
+    };
+    typename R4::V hr[2][16];
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) hr[half][i] = hload(half, i);
+    if (tid < 128) {
+        const int p = pos[tid];
+        grow[tid] = p >= 0 && p < N ? L.chunk[p] : -1;
+    }
+    __syncthreads();
     const int nchunks = (int)(dg / 64);
     auto load = [&](int c, uint32_t sa) {
         const uint32_t sb = sa + BinTC::A_BYTES;
@@ -189,26 +228,10 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_consta
         }
     };
     const uint32_t idesc = tc::idesc_bf16(128, nt, false, true);
-    constexpr bool kPrefetchH = sizeof(IN) == 2;
-    const uint32_t hbuf = base + BinTC::NS * BinTC::STAGE;
     bool ok = true;
     for (int c = 0; c < BinTC::NS - 1; ++c) {
         if (c < nchunks) load(c, base + (uint32_t)c * BinTC::STAGE);
         tc::cp_async_commit();
-        if (kPrefetchH && c == 0) {
-            // residual rows of this tile: [128][nt] bf16, row-major (zeros for empty rows)
-            const int nc = nt / 8;                               // 16-byte pieces per row, at most 32
-#pragma unroll 4
-            for (int e = tid; e < 128 * 32; e += 256) {
-                const int r = e >> 5, ch = e & 31;
-                const int p = pos[r];
-                if (ch < nc) {
-                    const IN *src = H + (size_t)(p >= 0 ? p : 0) * dl + n0 + ch * 8;
-                    tc::cp_async16(hbuf + (uint32_t)(r * nt + ch * 8) * 2, src, p >= 0 ? 16u : 0u);
-                }
-            }
-            tc::cp_async_commit();
-        }
     }
     for (int c = 0; c < nchunks; ++c) {
         const int cn = c + BinTC::NS - 1;
@@ -236,50 +259,40 @@ __global__ void __launch_bounds__(256, 1) bin_gemm_tc_kernel(const __grid_consta
     ok = __syncthreads_and(ok) != 0;
     tc::fence_after_sync();
     if (ok) {
-        // TMEM -> shared tile [128][nt] (row stride 260 floats), then one coalesced row at a time
         tc::cp_async_wait<0>();
         __syncthreads();
-        float *tile = reinterpret_cast<float *>(smraw + (base - tc::smem_u32(smraw)));
-        constexpr int LDT = 260;
-        // warps w and w + 4 read the same 32 TMEM lanes, each half of the columns
-        const int lg = warp & 3, half = nt / 2;
+        float *tilep = reinterpret_cast<float *>(smraw + (base - tc::smem_u32(smraw)));
+        // per column half: TMEM -> shared tile [128][LDT] (warps w and w + 4 read the same 32 TMEM
+        // lanes, each half of the columns), then one coalesced row at a time with the residual added
+        const int lg = warp & 3;
         const int r = lg * 32 + lane;
-#pragma unroll 1
-        for (int c0 = (warp >> 2) * half; c0 < (warp >> 2) * half + half; c0 += 16) {
-            float v[16];
-            tc::tmem_ld16(tbase + ((uint32_t)(lg * 32) << 16) + (uint32_t)c0, v);
-            float4 *d = reinterpret_cast<float4 *>(tile + r * LDT + c0);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
-        __syncthreads();
-        const int nvec = nt / 8;                                   // 8 columns per lane
+        for (int half = 0; half < 2; ++half) {
+            if (half * 128 >= nt) break;
+            const int w = min(128, nt - half * 128);             // 64 or 128 columns
+            const int cw = w / 2, cs = (warp >> 2) * cw;
 #pragma unroll 1
-        for (int rr = warp; rr < 128; rr += 8) {
-            const int p = pos[rr];
-            if (p < 0 || !dcheck(p < N, st)) continue;
-            for (int c8 = lane; c8 < nvec; c8 += 32) {
-                const float *t = tile + rr * LDT + c8 * 8;
-                const float4 a0 = *reinterpret_cast<const float4 *>(t);
-                const float4 a1 = *reinterpret_cast<const float4 *>(t + 4);
-                float h[8];
-                const IN *hrow = H + (size_t)p * dl + n0 + c8 * 8;
-                if (kPrefetchH) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(smraw + (hbuf - tc::smem_u32(smraw)) +
-                                                                     (size_t)(rr * nt + c8 * 8) * 2);
-                    const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&u);
+            for (int c0 = 0; c0 < cw; c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tbase + ((uint32_t)(lg * 32) << 16) + (uint32_t)(half * 128 + cs + c0), v);
+                float4 *d = reinterpret_cast<float4 *>(tilep + r * BinTC::LDT + cs + c0);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) h[i] = __bfloat162float(hb[i]);
-                } else {
-                    const float4 f0 = *reinterpret_cast<const float4 *>(hrow);
-                    const float4 f1 = *reinterpret_cast<const float4 *>(hrow + 4);
-                    h[0] = f0.x; h[1] = f0.y; h[2] = f0.z; h[3] = f0.w;
-                    h[4] = f1.x; h[5] = f1.y; h[6] = f1.z; h[7] = f1.w;
-                }
-                float4 *dst = reinterpret_cast<float4 *>(S + (size_t)p * dl + n0 + c8 * 8);
-                dst[0] = make_float4(a0.x + h[0], a0.y + h[1], a0.z + h[2], a0.w + h[3]);
-                dst[1] = make_float4(a1.x + h[4], a1.y + h[5], a1.z + h[6], a1.w + h[7]);
+                for (int q = 0; q < 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int rr = warp + 8 * i;
+                const int p = pos[rr];
+                if (p >= 0 && dcheck(p < N, st) && lane * 4 < w) {
+                    const float4 a = *reinterpret_cast<const float4 *>(tilep + rr * BinTC::LDT + lane * 4);
+                    float h[4];
+                    R4::unpack(hr[half][i], h);
+                    *reinterpret_cast<float4 *>(S + (size_t)p * dl + n0 + half * 128 + lane * 4) =
+                        make_float4(a.x + h[0], a.y + h[1], a.z + h[2], a.w + h[3]);
+                }
+            }
+            __syncthreads();                                     // the tile is rewritten by the next half
         }
     }
     tc::fence_before_sync();
@@ -306,14 +319,16 @@ inline dbc_status launch(const void *G, int64_t d_g, const void *H, int dtype, c
     dim3 g((unsigned)((N + 127) / 128 + nbins), (unsigned)((d_l + 255) / 256));
     if (dtype == DBC_BF16) {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)BinTC::smem<__nv_bfloat16>());
-        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 256, BinTC::smem<__nv_bfloat16>(), s>>>(
+                             (int)BinTC::SMEM);
+        // two CTAs per SM need the whole shared-memory carveout
+        cudaFuncSetAttribute(bin_gemm_tc_kernel<__nv_bfloat16>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        bin_gemm_tc_kernel<__nv_bfloat16><<<g, 256, BinTC::SMEM, s>>>(
             tmW, static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const __nv_bfloat16 *>(H), d_l, nbins, L,
             S, N, dev_status);
     } else {
         cudaFuncSetAttribute(bin_gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)BinTC::smem<float>());
-        bin_gemm_tc_kernel<float><<<g, 256, BinTC::smem<float>(), s>>>(
+                             (int)BinTC::SMEM);
+        bin_gemm_tc_kernel<float><<<g, 256, BinTC::SMEM, s>>>(
             tmW, static_cast<const __nv_bfloat16 *>(G), d_g, static_cast<const float *>(H), d_l, nbins, L, S, N,
             dev_status);
     }
