@@ -25,22 +25,27 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const uint4 *__r
                                                                 int64_t total, uint4 *__restrict__ Z, int32_t *st) {
     __shared__ int64_t s_offs[kOffsCache];
     const bool cached = rows + 1 <= kOffsCache;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kGatherThreads / 32);
+    const int64_t k_first = ((int64_t)blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp;
+    // the first step's boundary index is loaded together with the offsets cache (it does not
+    // depend on the row)
+    int64_t t_next = lane < kRowsPerWarp && k_first + lane < total ? idx[k_first + lane] : 0;
     if (cached)
         for (int64_t i = threadIdx.x; i <= rows; i += blockDim.x) s_offs[i] = idx_offsets[i];
     __syncthreads();
     const int64_t *offs = cached ? s_offs : idx_offsets;
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (kGatherThreads / 32);
-    for (int64_t k0 = ((int64_t)blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5)) * kRowsPerWarp; k0 < total;
-         k0 += warps * kRowsPerWarp) {
+    for (int64_t k0 = k_first; k0 < total; k0 += warps * kRowsPerWarp) {
         // source row start (in vectors) of chunk k0 + lane, or -1 (out of range / bad index)
         int64_t src = -1;
+        const int64_t t = t_next;
+        const int64_t kn = k0 + warps * kRowsPerWarp + lane;
+        if (lane < kRowsPerWarp && kn < total) t_next = idx[kn];
         if (lane < kRowsPerWarp && k0 + lane < total) {
             const int64_t k = k0 + lane;
             const int64_t r = find_row(offs, rows, k);
             int64_t a, n;
             row_bounds(offsets, r, T, a, n);
-            const int64_t t = idx[k];
             if (t < 0 || t >= n) flag(st, DBC_ERR_BOUNDS);
             else src = (a + t) * vec_per_row;
         }

@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(256, 1) gram_tma_kernel(const __grid_constant_
                 : "memory");
         }
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        // shared memory must outlive the stores' reads of it; the writes complete with the kernel
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
     tc::fence_before_sync();
     __syncthreads();

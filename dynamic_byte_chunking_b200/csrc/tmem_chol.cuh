@@ -652,7 +652,9 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                     }
                     cbar();
                 }
-                if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // region reused next
+                // the region is reused next: the stores must have read it (their writes may still be in
+                // flight; they are complete when the kernel is)
+                if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                 cbar();
             }
         }
