@@ -613,8 +613,11 @@ __global__ void __launch_bounds__(TmemChol::NT, 1) tmem_chol_kernel(
                 for (int q = 0; q < D / 64; ++q) {
                     const uint32_t stgb = region + (uint32_t)(q & 1) * (3u * 256u * 128u);
                     uint8_t *stg = smraw + (stgb - tc::smem_u32(smraw));
+                    // rows at or below the chunk's end hold zeros here and are not stored (warp-uniform:
+                    // a warp owns 32 consecutive rows)
+                    const bool live_q = row < (q + 1) * 64;
 #pragma unroll 1
-                    for (int h = 0; h < 4; ++h) {
+                    for (int h = 0; h < (live_q ? 4 : 0); ++h) {
                         float v16[16];
                         tc::tmem_ld16(trow + (uint32_t)(q * 64 + h * 16), v16);
 #pragma unroll
