@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--impl", default="dbc", choices=["dbc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-lanes", type=int, default=2,
+                    help="streams (each with its own buffers) that the end-to-end steps rotate over")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the device steps with eager launches instead of CUDA-graph replays")
     ap.add_argument("--rows", action="store_true",
@@ -692,8 +694,8 @@ def main():
 
     # ---- end to end through host buffers: every step copies its H from pinned host memory to the
     # device, runs the path through the API and reads (idx, Z, S) back into pinned host memory.  Steps
-    # alternate between two lanes, each with its own stream and buffers, so one step's device-to-host
-    # copies overlap the next step's host-to-device copy and compute (full-duplex copy engines).
+    # rotate over --e2e-lanes lanes, each with its own stream and buffers, so one step's device-to-host
+    # copies overlap the next steps' host-to-device copies and compute (full-duplex copy engines).
     e2e = None
     if args.e2e_steps > 0:
         class Lane:
@@ -727,10 +729,11 @@ def main():
                     self.o_Z.copy_(self.Z, non_blocking=True)
                     self.o_S.copy_(self.S, non_blocking=True)
 
-        lanes = [Lane(), Lane()]
+        nl = max(1, args.e2e_lanes)
+        lanes = [Lane() for _ in range(nl)]
         torch.cuda.synchronize()
-        for k in range(4):                    # warm-up of both lanes
-            lanes[k % 2].step()
+        for k in range(2 * nl):               # warm-up of every lane
+            lanes[k % nl].step()
         torch.cuda.synchronize()
         main_s = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -738,7 +741,7 @@ def main():
         for ln in lanes:
             ln.s.wait_event(e0)
         for k in range(args.e2e_steps):
-            lanes[k % 2].step()
+            lanes[k % nl].step()
         for ln in lanes:
             ev = torch.cuda.Event()
             ev.record(ln.s)
@@ -754,8 +757,8 @@ def main():
                "h2d_bytes_per_step": int(H_host.numel() * 2),
                "d2h_bytes_per_step": int(ln.o_idx.numel() * 8 + ln.o_Z.numel() * 2 + ln.o_S.numel() * 4),
                "ms_per_step": ms_e2e,
-               "pipelining": "two lanes (streams) alternate steps: device-to-host copies of one step overlap the "
-                             "next step's host-to-device copy and compute"}
+               "pipelining": f"{nl} lanes (streams) take steps in turn: device-to-host copies of one step overlap "
+                             "the next steps' host-to-device copies and compute"}
         del lanes
 
     torch.cuda.synchronize()
