@@ -124,6 +124,25 @@ def test_small_ragged_edge_lengths():
     _full_rows(w, True, name="edges")
 
 
+def test_new_directions_late_in_row():
+    # the first 1024 positions of each row span a 16-dimensional subspace, the rest every direction:
+    # the whitened rows of the segment at 1024 are large again (|y|^2 in the hundreds), so the
+    # in-segment Gram must take all six piece products there, not only in a row's first segments
+    d, T, r = 256, 2048, 16
+    rng = np.random.default_rng(11)
+    rows = []
+    for _ in range(2):
+        U = np.linalg.qr(rng.standard_normal((d, r)))[0]
+        low = rng.standard_normal((1024, r)) @ U.T / 4
+        full = rng.standard_normal((T - 1024, d)) / 16
+        rows.append(np.concatenate([low, full]))
+    Hb = workloads.bf16_bits(np.concatenate(rows).astype(np.float32))
+    offs = np.array([0, T, 2 * T], dtype=np.int64)
+    w = workloads.Workload("late-directions", "bf16", d, 0.5, offs, workloads.bf16_to_f32(Hb), Hb,
+                           np.full(2, T // 4, dtype=np.int64))
+    _full_rows(w, False, name="late-directions")
+
+
 def test_small_ragged_family():
     w = workloads.make("ragged", rows=7, T_range=(300, 2500), weights=False)
     _full_rows(w, True, name="small-ragged")
