@@ -318,6 +318,22 @@ def _time(fn, reps, flush, stream):
     return float(np.median(ts))
 
 
+def _time_graph(fn, reps, flush, stream):
+    """As _time, with fn captured once in a CUDA graph and replayed (kernel time without the host's
+    per-call launch cost)."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = _time(g.replay, reps, flush, stream)
+    del g
+    return ms
+
+
 def run_rows(args):
     """Each row of the hot path timed on the workload family it is specified on."""
     import torch
@@ -370,7 +386,7 @@ def run_rows(args):
             emit("NEXT-2 streaming coding rate (blocks of 256)", fam, ms, positions_per_s=N / (ms * 1e-3),
                  blocks=len(blocks), us_per_block=ms * 1e3 / len(blocks), tflops=fl / (ms * 1e-3) / 1e12)
             # latency of the smallest block: one new position per stream, 64 calls in a row mid-sequence
-            t_mid = 4096
+            t_mid = T // 2                       # mid-sequence, with 256 positions after it
             ones = [Hs[:, t:t + 1, :].contiguous() for t in range(t_mid, t_mid + 64)]
             ws1 = torch.empty(max(dbc.chunk_coding_rate_stream_workspace(rows, 1, t, d) for t in range(t_mid, t_mid + 64)),
                               dtype=torch.uint8, device=dev)
@@ -380,10 +396,30 @@ def run_rows(args):
                 for j, b in enumerate(ones):
                     dbc.chunk_coding_rate_stream(b, w.eps2, state, t_mid + j, dR=dR1, workspace=ws1)
 
-            ms1 = _time(byte_steps, args.reps, flush, stream)
+            ms1 = _time_graph(byte_steps, args.reps, flush, stream)
+            ms1e = _time(byte_steps, args.reps, flush, stream)
             emit("NEXT-2 streaming coding rate (one position per call)", fam, ms1, calls=len(ones),
-                 us_per_call=ms1 * 1e3 / len(ones), streams=rows)
-            del blocks, state, dRs, wss, ones, ws1, dR1
+                 us_per_call=ms1 * 1e3 / len(ones), us_per_call_eager=ms1e * 1e3 / len(ones), streams=rows,
+                 launch="graph")
+            # the per-position recursion (carried inverse factor): the same 64 one-position calls, and
+            # 256 positions in one call
+            Bst = dbc.step_state(rows, d, device=dev)
+
+            def step_calls():
+                for b in ones:
+                    dbc.chunk_coding_rate_step(b, w.eps2, Bst, dR=dR1)
+
+            ms2 = _time_graph(step_calls, args.reps, flush, stream)
+            ms2e = _time(step_calls, args.reps, flush, stream)
+            emit("NEXT-2 per-position recursion (one position per call)", fam, ms2, calls=len(ones),
+                 us_per_call=ms2 * 1e3 / len(ones), us_per_call_eager=ms2e * 1e3 / len(ones), streams=rows,
+                 launch="graph")
+            blk256 = Hs[:, t_mid:t_mid + 256, :].contiguous()
+            dR256 = torch.empty(rows * 256, dtype=torch.float32, device=dev)
+            ms3 = _time(lambda: dbc.chunk_coding_rate_step(blk256, w.eps2, Bst, dR=dR256), args.reps, flush, stream)
+            emit("NEXT-2 per-position recursion (256 positions per call)", fam, ms3, streams=rows,
+                 us_per_position=ms3 * 1e3 / 256, positions_per_s=rows * 256 / (ms3 * 1e-3))
+            del blocks, state, dRs, wss, ones, ws1, dR1, Bst, blk256, dR256
         if w.dtype == "bf16":
             # NEXT-4: the encoder's Canon layer (causal depthwise conv, k = 4) alone and chained with the chunker
             gen = np.random.default_rng(11)

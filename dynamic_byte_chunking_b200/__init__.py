@@ -26,7 +26,7 @@ from typing import Optional
 __all__ = [
     "DbcError", "lib", "lib_path", "version", "status_string", "launch_count",
     "chunk_coding_rate", "chunk_coding_rate_workspace", "chunk_coding_rate_stream",
-    "chunk_coding_rate_stream_workspace", "chunk_topk_select",
+    "chunk_coding_rate_stream_workspace", "chunk_coding_rate_step", "step_state", "chunk_topk_select",
     "chunk_gather", "chunk_upsample", "chunk_upsample_workspace", "chunk_upsample_noalloc",
     "chunk_upsample_backward", "chunk_upsample_backward_workspace", "chunk_gather_backward",
     "hnet_route", "hnet_route_workspace", "chunk", "canon_conv1d", "chunk_coding_rate_canon",
@@ -53,6 +53,7 @@ _SIGS = {
     "chunk_coding_rate": (_int, [_vp, _int, _vp, _i64, _i64, _i64, _i64, _f32, _vp, _vp, _sz, _vp, _vp]),
     "chunk_coding_rate_stream_workspace": (_sz, [_i64, _i64, _i64, _i64]),
     "chunk_coding_rate_stream": (_int, [_vp, _int, _i64, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "chunk_coding_rate_step": (_int, [_vp, _int, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _vp]),
     "chunk_topk_select_workspace": (_sz, [_i64]),
     "chunk_topk_select": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "chunk_gather": (_int, [_vp, _int, _vp, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp,
@@ -215,6 +216,32 @@ def chunk_coding_rate_stream(H, eps2: float, state, t0: int, *, dR=None, workspa
     rc = lib().chunk_coding_rate_stream(_ptr(H2), _dtype_code(H2), streams, n, d, int(t0), float(eps2), _ptr(state),
                                         _ptr(dR), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
     _check("chunk_coding_rate_stream", rc)
+    return dR
+
+
+def step_state(streams: int, d: int, device="cuda"):
+    """Per-byte stream state of new streams: the identity in fp32 [streams, d, d]."""
+    torch = _torch()
+    return torch.eye(d, dtype=torch.float32, device=device).repeat(streams, 1, 1).contiguous()
+
+
+def chunk_coding_rate_step(H, eps2: float, B_state, *, dR=None, dev_status=None, stream=None):
+    """dR (fp32 [streams * n]) of n new positions per stream ([streams, n, d], fp32 or bf16, d <= 256),
+    one position at a time from the carried factor ``B_state`` (fp32 [streams, d, d], the identity for
+    new streams, see ``step_state``), which is advanced in place."""
+    torch = _torch()
+    _require_cuda(H, B_state)
+    if H.dim() != 3:
+        raise ValueError("H must be [streams, n, d]")
+    streams, n, d = H.shape
+    if B_state.dtype != torch.float32 or tuple(B_state.shape) != (streams, d, d) or not B_state.is_contiguous():
+        raise TypeError("B_state must be a contiguous float32 [streams, d, d] tensor")
+    H2 = H.contiguous()
+    if dR is None:
+        dR = torch.empty(streams * n, dtype=torch.float32, device=H.device)
+    rc = lib().chunk_coding_rate_step(_ptr(H2), _dtype_code(H2), streams, n, d, float(eps2), _ptr(B_state),
+                                      _ptr(dR), _ptr(dev_status), _stream(stream))
+    _check("chunk_coding_rate_step", rc)
     return dR
 
 

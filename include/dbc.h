@@ -133,6 +133,37 @@ DBC_API dbc_status chunk_coding_rate_stream(const void *H, int dtype, int64_t st
                                             size_t ws_bytes, int32_t *dev_status, dbc_stream_t stream);
 
 /* -------------------------------------------------------------------------
+ * chunk_coding_rate_step -- the marginal coding rate of streams, one new
+ * position at a time (the per-byte recursion).
+ *
+ * ByteFlow (summary "Prerequisites: lossy coding rate", "Method steps",
+ * stage 2, "Limitations and improvements" first point, and "Weaknesses of the
+ * independent analysis": an incremental per-byte update).  Each stream
+ * carries B = L^{-T}, the inverse transposed Cholesky factor of
+ * M = I + c sum h_i h_i^T over everything it has seen (c = d / eps2).  For
+ * each new position h, in order: w = sqrt(c) B^T h, dR = 1/2 log(1 + |w|^2),
+ * and B becomes the factor of M + c h h^T (an O(d^2) rank-one update of B).
+ * The values equal the whole sequence's dR (same definition as
+ * chunk_coding_rate) up to fp32 rounding, for any split of the stream into
+ * calls; a call costs O(n d^2) on one SM per stream, so long blocks are
+ * cheaper through chunk_coding_rate_stream.
+ *
+ * H        fp32 or bf16 (dtype) [streams, n, d] the new positions; d a
+ *          multiple of 4, at most 256.
+ * B_state  in/out fp32 [streams, d, d] row-major, 16-byte aligned: the upper
+ *          triangle (with the diagonal) holds B before and after the call; the
+ *          strictly lower triangle is not used and not written.  A new stream
+ *          starts from the identity (M = I).  Caller-owned.
+ * dR       out fp32 [streams, n].
+ * Errors: INVALID_ARG (NULL, negative sizes, eps2 <= 0, misaligned state),
+ * UNSUPPORTED (dtype, d > 256 or not a multiple of 4), CUDA; device flag
+ * NONFINITE.
+ * ------------------------------------------------------------------------- */
+DBC_API dbc_status chunk_coding_rate_step(const void *H, int dtype, int64_t streams, int64_t n, int64_t d,
+                                          float eps2, float *B_state, float *dR, int32_t *dev_status,
+                                          dbc_stream_t stream);
+
+/* -------------------------------------------------------------------------
  * chunk_topk_select -- boundary positions per row.
  *
  * ByteFlow (notes "Key design 2"; summary stage 2): position 0 (BOS) is always

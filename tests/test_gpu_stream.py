@@ -70,3 +70,56 @@ def test_stream_windowed_selection():
     ridx, rio = topk_select_rows(dRn, np.arange(nwin + 1, dtype=np.int64) * W, k)
     assert np.array_equal(io.cpu().numpy(), rio)
     assert np.array_equal(idx.cpu().numpy(), ridx)
+
+
+# ---------------------------------------------------------------- per-position recursion
+@pytest.mark.parametrize("fam,S,blocks", [
+    ("byteflow", 3, [1, 1, 3, 64, 250, 381]),       # d = 256, bf16, one-position calls first
+    ("byteflow", 2, [256] * 16),                     # 4096 rank-one updates of the carried factor
+    ("bytegen", 2, [1, 511, 608]),                   # structured rows (whole 32-byte market events)
+    ("tiny", 2, [1, 7, 300]),                        # d = 64, fp32
+])
+def test_step_equals_whole_sequence(fam, S, blocks):
+    import torch
+    import dynamic_byte_chunking_b200 as dbc
+    T = sum(blocks)
+    w = workloads.make(fam, rows=S, T=T, weights=False)
+    if w.dtype == "bf16":
+        H = bf16_dev(w.H_bits).view(S, T, w.d)
+    else:
+        H = torch.from_numpy(np.ascontiguousarray(w.H_bits)).cuda().view(S, T, w.d)
+    B = dbc.step_state(S, w.d)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs, t0 = [], 0
+    for n in blocks:
+        outs.append(dbc.chunk_coding_rate_step(H[:, t0:t0 + n, :], w.eps2, B, dev_status=st).view(S, n))
+        t0 += n
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    dR = torch.cat(outs, dim=1).cpu().numpy()
+    ref = dR_rank1(w.H, w.offsets, w.eps2).reshape(S, T)
+    for r in range(S):
+        check_dR(dR[r], ref[r], w.dtype, f"step-{fam}-{len(blocks)}calls/row{r}")
+    # the carried factor: B^T M B = I for the M of everything fed (M = I + c X^T X)
+    X = np.asarray(w.H, dtype=np.float64).reshape(S, T, w.d)
+    c = w.d / w.eps2
+    Bh = np.triu(B.cpu().numpy().astype(np.float64))
+    for r in range(S):
+        M = np.eye(w.d) + c * X[r].T @ X[r]
+        E = Bh[r].T @ M @ Bh[r] - np.eye(w.d)
+        rel = np.abs(E).max()
+        record(f"step-{fam}-{len(blocks)}calls/row{r}:BtMB", max_abs=rel)
+        assert rel <= 1e-2
+
+
+def test_step_leaves_lower_triangle_alone():
+    import torch
+    import dynamic_byte_chunking_b200 as dbc
+    w = workloads.make("tiny", rows=1, T=40, weights=False)
+    H = torch.from_numpy(np.ascontiguousarray(w.H_bits)).cuda().view(1, 40, w.d)
+    B = dbc.step_state(1, w.d)
+    low = torch.tril(torch.full((w.d, w.d), 7.0, device="cuda"), diagonal=-1)
+    B += low
+    dbc.chunk_coding_rate_step(H, w.eps2, B)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.tril(B[0], diagonal=-1), low)
