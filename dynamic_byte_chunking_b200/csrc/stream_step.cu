@@ -22,50 +22,77 @@
 //
 // so the update of the whole factor is O(d^2) per position with one fused
 // multiply-add on each row's serial chain.  One CTA per stream keeps the
-// upper triangle of B in shared memory (d(d+1)/2 floats, 129 KB at d = 256)
-// for all the call's positions; thread k owns column k for w and row k for
-// the update.
+// upper triangle of B in shared memory (158 KB at d = 256, layout below) for
+// all the call's positions, moving it in and out as one bulk copy per row;
+// thread k owns column k for w and row k for the update.
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace dbc {
 namespace ss {
 
 constexpr int kThreads = 256;      // = the largest d
 constexpr int kMaxD = 256;
+constexpr int kSkew = 28;          // spare floats per row: a 16-byte-step shift of up to 7 pieces
 
-// Offset of row i of the packed upper triangle (row i holds columns i .. d-1).
-__device__ __forceinline__ int row_start(int i, int d) { return i * d - (i * (i - 1)) / 2; }
+// Shared layout of the carried factor: row i holds columns (i & ~3) .. d-1 (len(i) = d - (i & ~3)
+// floats, a whole number of 16-byte pieces, so each row moves as one bulk copy; the up to three
+// entries left of the diagonal are carried along untouched).  Rows are laid out back to back with
+// kSkew spare floats each (row_base), and row i starts some whole pieces into its room, chosen so
+// that its update thread (thread i: lane i % 32, with the neighbouring rows of similar length in
+// the same warp) meets a bank no other lane of its warp meets: at every step the 32 lanes' entries
+// (row i, column i + step) fall in 32 different banks.
+__device__ __forceinline__ int row_len(int i, int d) { return d - (i & ~3); }
+__device__ __forceinline__ int row_base(int i, int d) {
+    const int q = i >> 2, r = i & 3;
+    return i * (d + kSkew) - 4 * (2 * q * (q - 1) + r * q);
+}
+__device__ __forceinline__ int row_start(int i, int d) {
+    const int b = row_base(i, d);
+    return b + 4 * ((((i >> 2) & 7) - (b >> 2)) & 7);
+}
 
-inline size_t smem_bytes(int d) { return (size_t)d * (d + 1) / 2 * sizeof(float); }
+inline size_t smem_bytes(int d) {
+    const int q = d >> 2;
+    return (size_t)(d * (d + kSkew) - 8 * q * (q - 1)) * sizeof(float);
+}
 
 template <class IN>
 __global__ void __launch_bounds__(kThreads) step_kernel(const IN *__restrict__ H, int64_t n, int d, float sqrt_c,
                                                         float *__restrict__ Bstate, float *__restrict__ dR,
                                                         int32_t *st) {
-    extern __shared__ float Bp[];                    // packed upper triangle of B
+    extern __shared__ __align__(16) float Bp[];
     // per column k of this position: (w_k, sqrt(beta_{k-1}/beta_k), beta_{k-1}/beta_k, w_k/beta_k)
     __shared__ float4 s_col[kMaxD];
-    __shared__ float s_h[kMaxD];
+    __shared__ __align__(16) float s_h[kMaxD];
+    __shared__ __align__(16) int s_off[kMaxD];       // s_off[i] + c = entry (i, c) for c >= (i & ~3)
     __shared__ float s_wsum[kThreads / 32];
+    __shared__ uint64_t mbar;
     const int k = threadIdx.x, lane = k & 31, warp = k >> 5;
     const int64_t s = blockIdx.x;
     float *B = Bstate + s * (int64_t)d * d;
-    // the carried factor's upper triangle: row i's entries i .. d-1 are contiguous in both layouts, so
-    // every element is one 4-byte asynchronous copy, all in flight at once (16-byte pieces through
-    // registers measured no faster)
-    {
-        const uint32_t sb = (uint32_t)__cvta_generic_to_shared(Bp);
-        int o = k;
-#pragma unroll 8
-        for (int i = 0; i < d; ++i) {
-            if (k >= i && k < d)
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sb + 4u * (uint32_t)o),
-                             "l"(B + (int64_t)i * d + k) : "memory");
-            o += d - 1 - i;
-        }
+    if (k < d) s_off[k] = row_start(k, d) - (k & ~3);
+    if (k == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    // the carried factor: one bulk copy per row (16-byte aligned on both sides), all in flight at once
+    if (k == 0) {
+        uint32_t bytes = 0;
+        for (int i = 0; i < d; ++i) bytes += 4u * (uint32_t)row_len(i, d);
+        tc::mbar_arrive_expect_tx(&mbar, bytes);
+    }
+    __syncthreads();
+    if (k < d)
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                         tc::smem_u32(Bp + row_start(k, d))),
+                     "l"(B + (int64_t)k * d + (k & ~3)), "r"(4u * (uint32_t)row_len(k, d)), "r"(tc::smem_u32(&mbar))
+                     : "memory");
+    bool ok = tc::mbar_wait(&mbar, 0, st);
+    if (!ok) ok = tc::mbar_wait(&mbar, 0, st);        // the copies land before the CTA may leave
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok) return;
     const IN *Hs = H + s * n * (int64_t)d;
     float h_next = k < d && n > 0 ? ld_f(Hs + k) : 0.f;
     for (int64_t t = 0; t < n; ++t) {
@@ -73,30 +100,26 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const IN *__restrict__ H
         if (k < d && !isfinite(hk)) flag(st, DBC_ERR_NONFINITE);
         if (k < d) s_h[k] = hk;
         if (k < d && t + 1 < n) h_next = ld_f(Hs + (t + 1) * d + k);
-        __syncthreads();                              // h in place; the factor (or the last update) complete
-        // w_k = sqrt(c) sum_{i <= k} B_ik h_i: column k of the packed rows (row i starts at
-        // row_start(i), so the entry moves by d - 1 - i from row i to row i + 1)
+        __syncthreads();                              // h in place; the last update complete
+        // w_k = sqrt(c) sum_{i <= k} B_ik h_i: column k, four rows per round (their offsets and h
+        // values as broadcast 16-byte loads), two rounds of loads before the multiply-adds
         float wk = 0.f;
         if (k < d) {
-            // eight rows per round, every load issued before the multiply-adds
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            int i = 0, off = k;                       // off = row_start(i) + (k - i)
+            int i = 0;
             for (; i + 8 <= k + 1; i += 8) {
-                float bv[8];
-                int o = off;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    bv[u] = Bp[o];
-                    o += d - 1 - (i + u);
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) acc[u] = fmaf(bv[u], s_h[i + u], acc[u]);
-                off = o;
+                const int4 o0 = *reinterpret_cast<const int4 *>(s_off + i);
+                const int4 o1 = *reinterpret_cast<const int4 *>(s_off + i + 4);
+                const float4 h0 = *reinterpret_cast<const float4 *>(s_h + i);
+                const float4 h1 = *reinterpret_cast<const float4 *>(s_h + i + 4);
+                const float b0 = Bp[o0.x + k], b1 = Bp[o0.y + k], b2 = Bp[o0.z + k], b3 = Bp[o0.w + k];
+                const float b4 = Bp[o1.x + k], b5 = Bp[o1.y + k], b6 = Bp[o1.z + k], b7 = Bp[o1.w + k];
+                acc[0] = fmaf(b0, h0.x, acc[0]); acc[1] = fmaf(b1, h0.y, acc[1]);
+                acc[2] = fmaf(b2, h0.z, acc[2]); acc[3] = fmaf(b3, h0.w, acc[3]);
+                acc[4] = fmaf(b4, h1.x, acc[4]); acc[5] = fmaf(b5, h1.y, acc[5]);
+                acc[6] = fmaf(b6, h1.z, acc[6]); acc[7] = fmaf(b7, h1.w, acc[7]);
             }
-            for (; i <= k; ++i) {
-                acc[0] = fmaf(Bp[off], s_h[i], acc[0]);
-                off += d - 1 - i;
-            }
+            for (; i <= k; ++i) acc[0] = fmaf(Bp[s_off[i] + k], s_h[i], acc[0]);
             wk = ((acc[0] + acc[1]) + (acc[2] + acc[3]) + ((acc[4] + acc[5]) + (acc[6] + acc[7]))) * sqrt_c;
         }
         // inclusive scan of w_k^2 over k: q_k = sum_{j <= k} w_j^2
@@ -124,17 +147,16 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const IN *__restrict__ H
         }
         if (k == 0) dR[s * n + t] = 0.5f * log1pf(total);
         __syncthreads();
-        // row k of B: x solves V x = b (b_j = 0 left of the diagonal, so the sum starts at k).  Four
-        // columns per group, the next group's loads before this group's stores (the entries differ).
-        // Lanes walk their own rows from their own diagonals: the rows' starts fall in different banks
-        // (a warp-aligned walk, with broadcast coefficients, measured slower)
+        // row my_row of B: x solves V x = b (b_j = 0 left of the diagonal, so the sum starts at the
+        // diagonal).  Four columns per group, the next group's loads before this group's stores.
         if (k < d) {
-            float *row = Bp + row_start(k, d) - k;    // row[j] = B_kj for j >= k
+            const int r0 = k;
+            float *row = Bp + s_off[r0];              // row[j] = B_(r0)j for j >= r0
             float sigma = 0.f;
-            const int ng = (d - k) / 4;               // whole groups of four columns
+            const int ng = (d - r0) / 4;
             float b[4], bn[4];
             float4 cl[4], cn[4];
-            int j = k;
+            int j = r0;
             if (ng > 0) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) { b[u] = row[j + u]; cl[u] = s_col[j + u]; }
@@ -164,27 +186,16 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const IN *__restrict__ H
             }
         }
     }
+    // back to the caller's rows, one bulk copy per row (the entries left of the diagonal that a row's
+    // first piece carries go back unchanged)
+    tc::fence_async_smem();
     __syncthreads();
-    // back to the caller's rows, eight rows per round with their shared loads first (the strictly
-    // lower triangle is not written)
-    {
-        int o = k;
-        for (int i0 = 0; i0 < d; i0 += 8) {
-            float v[8];
-            int oo = o;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u;
-                v[u] = (i < d && k >= i && k < d) ? Bp[oo] : 0.f;
-                oo += d - 1 - i;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u;
-                if (i < d && k >= i && k < d) B[(int64_t)i * d + k] = v[u];
-            }
-            o = oo;
-        }
+    if (k < d) {
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(B + (int64_t)k * d + (k & ~3)),
+                     "r"(tc::smem_u32(Bp + row_start(k, d))), "r"(4u * (uint32_t)row_len(k, d))
+                     : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
 }
 

@@ -152,8 +152,11 @@ DBC_API dbc_status chunk_coding_rate_stream(const void *H, int dtype, int64_t st
  *          multiple of 4, at most 256.
  * B_state  in/out fp32 [streams, d, d] row-major, 16-byte aligned: the upper
  *          triangle (with the diagonal) holds B before and after the call; the
- *          strictly lower triangle is not used and not written.  A new stream
- *          starts from the identity (M = I).  Caller-owned.
+ *          strictly lower triangle is not used and keeps its values (rows move
+ *          in 16-byte pieces, so up to three entries left of each diagonal are
+ *          read and written back unchanged).  A new stream starts from the
+ *          identity (M = I).  Caller-owned; not to be written by other work
+ *          while the call runs.
  * dR       out fp32 [streams, n].
  * Errors: INVALID_ARG (NULL, negative sizes, eps2 <= 0, misaligned state),
  * UNSUPPORTED (dtype, d > 256 or not a multiple of 4), CUDA; device flag
