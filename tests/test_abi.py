@@ -122,3 +122,22 @@ def test_stream_argument_errors_and_workspace(L):
     a = dbc.chunk_coding_rate_stream_workspace(4, 256, 1, 256)
     b = dbc.chunk_coding_rate_stream_workspace(4, 256, 256, 256)
     assert a > b > 0
+
+
+def test_step_argument_errors_return_before_launch(L):
+    f = L.chunk_coding_rate_step
+    dummy = ctypes.c_void_p(16)          # never dereferenced: every case returns before a launch
+    odd = ctypes.c_void_p(20)            # not 16-byte aligned
+    # dtype, d above 256 or not a multiple of 4
+    assert f(dummy, 7, 1, 1, 256, ctypes.c_float(0.5), dummy, dummy, None, None) == 2
+    assert f(dummy, 1, 1, 1, 260, ctypes.c_float(0.5), dummy, dummy, None, None) == 2
+    assert f(dummy, 1, 1, 1, 30, ctypes.c_float(0.5), dummy, dummy, None, None) == 2
+    # negative sizes, eps2 <= 0, missing buffers, a misaligned state
+    assert f(dummy, 1, -1, 1, 256, ctypes.c_float(0.5), dummy, dummy, None, None) == 1
+    assert f(dummy, 1, 1, 1, 256, ctypes.c_float(0.0), dummy, dummy, None, None) == 1
+    assert f(None, 1, 1, 1, 256, ctypes.c_float(0.5), dummy, dummy, None, None) == 1
+    assert f(dummy, 1, 1, 1, 256, ctypes.c_float(0.5), None, dummy, None, None) == 1
+    assert f(dummy, 1, 1, 1, 256, ctypes.c_float(0.5), odd, dummy, None, None) == 1
+    # no streams or no positions: nothing to do
+    assert f(None, 1, 0, 1, 256, ctypes.c_float(0.5), None, None, None, None) == 0
+    assert f(None, 1, 3, 0, 256, ctypes.c_float(0.5), None, None, None, None) == 0
