@@ -120,10 +120,11 @@ __global__ void __launch_bounds__(256) scatter_kernel(int64_t N, int nbins, Layo
 // scatters the rows back to their positions.  Two stages of 48 KB keep the CTA
 // small enough for two per SM (with bf16 h), so one CTA's epilogue stores run
 // under the other's loads and MMAs.  The tile's residual values are loaded into
-// registers as soon as its positions are known, before anything else: each CTA
-// lives for one tile, so the DRAM reads it keeps in flight are what bounds the
-// kernel (issuing the second column half's loads only during the first half's
-// stores cost a quarter of the time on the ragged batch).
+// registers early: the first column half's as soon as the positions are known,
+// the second half's right after the first K chunk's operand loads (so those go
+// out first).  Each CTA lives for one tile, so the DRAM reads it keeps in flight
+// are what bounds the kernel (issuing the second half's loads only during the
+// first half's stores cost a quarter of the time on the ragged batch).
 struct BinTC {
     static constexpr int NS = 2;
     static constexpr uint32_t A_BYTES = 128 * 128;             // 128 rows x 64 K, K-major
@@ -188,8 +189,9 @@ __global__ void __launch_bounds__(256, sizeof(IN) == 2 ? 2 : 1)
     tc::fence_after_sync();
     const uint32_t tbase = tmem_base;
     // Residual of row (warp + 8 i), columns half * 128 + lane * 4 .. +3 (zeros for empty rows and
-    // columns past the tile): all of the tile's residual loads are issued here, before the chunk
-    // rows are looked up, and stay in flight through the MMAs
+    // columns past the tile): the first half's loads are issued here, before the chunk rows are
+    // looked up, the second half's after the first operand loads; they stay in flight through the
+    // MMAs
     using R4 = Res4<IN>;
     auto hload = [&](int half, int i) {
         typename R4::V v{};
@@ -200,9 +202,7 @@ __global__ void __launch_bounds__(256, sizeof(IN) == 2 ? 2 : 1)
     };
     typename R4::V hr[2][16];
 #pragma unroll
-    for (int half = 0; half < 2; ++half)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) hr[half][i] = hload(half, i);
+    for (int i = 0; i < 16; ++i) hr[0][i] = hload(0, i);
     if (tid < 128) {
         const int p = pos[tid];
         grow[tid] = p >= 0 && p < N ? L.chunk[p] : -1;
@@ -233,6 +233,8 @@ __global__ void __launch_bounds__(256, sizeof(IN) == 2 ? 2 : 1)
         if (c < nchunks) load(c, base + (uint32_t)c * BinTC::STAGE);
         tc::cp_async_commit();
     }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) hr[1][i] = hload(1, i);
     for (int c = 0; c < nchunks; ++c) {
         const int cn = c + BinTC::NS - 1;
         if (cn < nchunks) {
